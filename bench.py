@@ -1,0 +1,403 @@
+"""Throughput of exact attention (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload long_ctx] [--seq N] [--no-cpu-baseline] [--e2e-steps E]
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+the forward kernel, then the three backward kernels (D preprocess, main,
+dQ convert), all through the library's C ABI.  The default workload is the
+long-context causal bf16 attention layer B=1, H=16, N=16384, d=128 (Q, K, V
+scaled by 0.5), the configuration the headline tensor-roofline target is
+quoted on.  Flops are algorithmic: forward 4*B*H*N*N*d, halved for causal;
+backward 2.5x that.
+
+Rank 0 prints ONE JSON line.  For N > 1 (torchrun, one process per GPU) every
+rank runs an independent replica of the workload: the path has no exchange
+step, so there is no collective on the data path; the timing is the max over
+ranks (an all-reduce of the elapsed time only).
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on a
+bounded sample of the same workload on the host cores, and prints the same
+line with "impl": "reference".
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s on 1 B200 and fraction of dense BF16/FP16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+# dram__bytes_read.sum + dram__bytes_write.sum of one bwd_main_kernel launch
+# (bf16, causal, d=128) from an ncu capture; None until captured for the
+# current kernel.  Keyed by (N, H) of the captured case.
+BWD_MAIN_TRAFFIC = None
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="long_ctx")
+    p.add_argument("--seq", type=int, default=None, help="override the sequence length (profiling runs)")
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def get_workload(name, seq):
+    import dataclasses
+    from exact_attention_150_b200 import workloads
+    w = workloads.by_name(name)
+    if seq is not None:
+        w = dataclasses.replace(w, N=seq, name=f"{w.name}_N{seq}")
+    return w
+
+
+def dist_info():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank processes `steps` steps of its replica."""
+    return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
+def sample_flops(w, rows) -> float:
+    """Algorithmic fwd+bwd flops of query rows `rows` (absolute indices) of one head."""
+    keys = sum((r + 1) if w.causal else w.N for r in rows)
+    return 4.0 * w.d * keys * 3.5  # forward (4 d per visible key) plus backward at 2.5x
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        time.sleep(0.2)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        else:
+            self.lines = []
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample_run(w, q, k, v, do, rows_count: int):
+    """One fp64 oracle forward + backward on the last `rows_count` query rows
+    of head (0, 0) against all keys.  Returns (seconds, flops, description)."""
+    import oracle
+    import torch
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    n = w.N
+    r0 = n - rows_count
+    qs, dos = f64(q[0, 0, r0:]), f64(do[0, 0, r0:])
+    ks, vs = f64(k[0, 0]), f64(v[0, 0])
+    t0 = time.perf_counter()
+    oracle.forward(qs, ks, vs, w.scale, w.causal, q_offset=r0)
+    oracle.backward(qs, ks, vs, dos, w.scale, w.causal, q_offset=r0)
+    dt = time.perf_counter() - t0
+    desc = (f"fp64 oracle forward+backward of query rows [{r0},{n}) of head (0,0) against all {n} keys "
+            f"({rows_count} of {w.B * w.H * n} rows of the workload)")
+    return dt, sample_flops(w, range(r0, n)), desc
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = [x for x in threadpool_info() if x.get("user_api") == "blas"]
+        if info:
+            return int(max(x.get("num_threads", 1) for x in info))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- arms
+
+def config_of(w, world):
+    return {"workload": w.label(), "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "passes": "fwd+bwd" if w.backward else "fwd", "input_scale": w.input_scale,
+            "l2": "no flush: inputs larger than the 126 MB L2 (Q, K, V, dO of %d MB each)"
+                  % (w.B * w.H * w.N * w.d * 2 // 2**20),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_info()
+    if rank != 0:
+        return 0
+    from exact_attention_150_b200 import workloads
+    w = get_workload(args.workload, args.seq)
+    q, k, v, do = workloads.make_inputs(w, with_grad=True)
+    rows = 512
+    times, flops = [], 0.0
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        dt, fl, desc = oracle_sample_run(w, q, k, v, do, rows)
+        if i >= args.warmup:
+            times.append(dt)
+            flops = fl
+    total = sum(times)
+    value = flops * len(times) / total / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": "each step: " + desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    rank, world, local_rank = dist_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(device)
+
+    from exact_attention_150_b200 import native, workloads
+    native.load()
+    w = get_workload(args.workload, args.seq)
+    q_h, k_h, v_h, do_h = workloads.make_inputs(w, with_grad=True)
+    q, k, v, do = (t.to(device) for t in (q_h, k_h, v_h, do_h))
+    o = torch.empty_like(q)
+    lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(native.attn_bwd_workspace_bytes(w.B, w.H, w.N, w.N, w.d), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def fwd():
+        native.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+
+    def bwd(phase):
+        native.backward(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, dq=dq, dk=dk, dv=dv, workspace=ws,
+                        phase=phase)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fwd()
+        if not w.backward:
+            if ev is not None:
+                ev[1].record(stream)
+            return
+        if ev is not None:
+            ev[1].record(stream)
+        bwd(native.ATTN_BWD_PREPROCESS)
+        if ev is not None:
+            ev[2].record(stream)
+        bwd(native.ATTN_BWD_MAIN)
+        if ev is not None:
+            ev[3].record(stream)
+        bwd(native.ATTN_BWD_CONVERT)
+        if ev is not None:
+            ev[4].record(stream)
+
+    launches_per_step = 4 if w.backward else 1
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize(device)
+    native.device_status()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    native.device_status()
+    elapsed = start.elapsed_time(end)
+    max_ms = max_over_ranks(elapsed, world, device)
+
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    step_flops = w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)
+    value = aggregate(step_flops, args.steps, world, max_ms)
+    peaks, peak_src = load_peaks()
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    kernels = {"fwd_kernel": {"ms": fwd_ms, "tflops": w.fwd_flops() / fwd_ms / 1e9}}
+    if w.backward:
+        pre_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+        post_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
+        rows = w.B * w.H * w.N
+        kernels["bwd_pre_kernel"] = {"ms": pre_ms, "gbs": rows * (2 * w.d * 2 + 4 + 8 + 4 * w.d) / pre_ms / 1e6}
+        kernels["bwd_main_kernel"] = {"ms": main_ms, "tflops": w.bwd_flops() / main_ms / 1e9}
+        kernels["bwd_post_kernel"] = {"ms": post_ms, "gbs": rows * w.d * (4 + 2) / post_ms / 1e6}
+        dom_name, dom_ms, dom_flops = "bwd_main_kernel", main_ms, w.bwd_flops()
+    else:
+        dom_name, dom_ms, dom_flops = "fwd_kernel", fwd_ms, w.fwd_flops()
+    for name, kinfo in kernels.items():
+        if "tflops" in kinfo:
+            kinfo["frac"] = kinfo["tflops"] / peak_sus
+    achieved = dom_flops / dom_ms / 1e9
+    traffic = None
+    if BWD_MAIN_TRAFFIC is not None and dom_name == "bwd_main_kernel":
+        traffic = BWD_MAIN_TRAFFIC.get((w.N, w.H))
+
+    # End to end through the public API: pinned host inputs -> device, the
+    # forward and backward calls, results -> pinned host, every step.
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = lambda t: t.pin_memory()
+        hq, hk, hv, hdo = (pin(t) for t in (q_h, k_h, v_h, do_h))
+        outs_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in outs_h)
+
+        def e2e_step():
+            for dst, src in ((q, hq), (k, hk), (v, hv), (do, hdo)):
+                dst.copy_(src, non_blocking=True)
+            fwd()
+            if w.backward:
+                bwd(native.ATTN_BWD_ALL)
+            for dst, src in zip(outs_h, (o, lse, dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(device)
+        if world > 1:
+            torch.distributed.barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize(device)
+        if world > 1:
+            torch.distributed.barrier()
+        native.device_status()
+        e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, device)
+        e2e = {"value": aggregate(step_flops, args.e2e_steps, world, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl, desc = oracle_sample_run(w, q_h, k_h, v_h, do_h, min(4096, w.N))
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": desc}
+
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp16",
+        "data": "synthetic: seeded i.i.d. N(0,1) Q, K, V, dO (x%g)" % w.input_scale,
+        "config": config_of(w, world),
+        "fwd_tflops": w.fwd_flops() / fwd_ms / 1e9,
+        "bwd_tflops": (w.bwd_flops() / (max_ms / args.steps - fwd_ms) / 1e9) if w.backward else None,
+        "kernels": kernels,
+        "roofline": {"kernel": dom_name, "bound": "tensor", "achieved": achieved, "peak": peak_sus,
+                     "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)"},
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

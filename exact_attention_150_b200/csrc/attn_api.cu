@@ -1,0 +1,228 @@
+// attn_api.cu -- the C ABI declared in include/attn.h: host-side argument
+// validation, TMA tensor-map construction and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "bwd_kernel.cuh"
+#include "fwd_kernel.cuh"
+
+namespace {
+
+using attn::kTile;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D view [rows][d] of a contiguous 16-bit tensor, read in boxes of 64
+// columns (128 bytes) x 128 rows with the 128-byte swizzle the MMA
+// descriptors expect.
+bool make_map(CUtensorMap* map, const void* base, long long rows, int d, bool bf16) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTile)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+attn_status check_common(int B, int H, int Nq, int Nk, int d, int causal, attn_dtype dtype) {
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_FP16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Nq % kTile != 0 || Nk % kTile != 0) return ATTN_ERR_UNSUPPORTED;
+  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
+  const long long bh = static_cast<long long>(B) * H;
+  // TMA row coordinates and grid dimensions are 32-bit.
+  if (bh > 0x7fffffffLL || bh * Nq > 0x7fffffffLL || bh * Nk > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (Nq / (2 * kTile) + 1 > 65535 || Nk / kTile > 65535) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int D, bool BF16, bool CAUSAL>
+attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse,
+                       int BH, int Nq, int Nk, float scale_log2, cudaStream_t st) {
+  using L = attn::FwdLayout<D>;
+  auto kern = attn::fwd_kernel<D, BF16, CAUSAL>;
+  if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int pairs = (Nq / kTile + 1) / 2;
+  dim3 grid(BH, pairs);
+  kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, Nq, Nk, scale_log2, pairs);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool BF16, bool CAUSAL>
+attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                       const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv, float* ws,
+                       int BH, int Nq, int Nk, float scale, int phase, cudaStream_t st) {
+  using L = attn::BwdLayout<D>;
+  const long long qrows = static_cast<long long>(BH) * Nq;
+  float* dqacc = ws;
+  float* dvec = ws + qrows * D;
+  float* nlse2 = dvec + qrows;
+
+  if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_PREPROCESS) {
+    constexpr int kRowsPerBlock = 256 / (D / 8);
+    const long long pre_blocks = (qrows + kRowsPerBlock - 1) / kRowsPerBlock;
+    attn::bwd_pre_kernel<D, BF16><<<static_cast<unsigned>(pre_blocks), 256, 0, st>>>(
+        static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, dvec, nlse2, dqacc, qrows);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_MAIN) {
+    auto kern = attn::bwd_main_kernel<D, BF16, CAUSAL>;
+    if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
+    dim3 grid(BH, Nk / kTile);
+    kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, dqacc, static_cast<uint16_t*>(dk),
+                                       static_cast<uint16_t*>(dv), Nq, Nk, scale, scale * 1.4426950408889634f);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_CONVERT) {
+    const long long n8 = qrows * D / 8;
+    long long post_blocks = (n8 + 255) / 256;
+    if (post_blocks > 148LL * 16) post_blocks = 148LL * 16;
+    attn::bwd_post_kernel<BF16>
+        <<<static_cast<unsigned>(post_blocks), 256, 0, st>>>(dqacc, static_cast<uint16_t*>(dq), n8);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+template <int D, bool BF16>
+attn_status dispatch_fwd_causal(int causal, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                void* o, float* lse, int BH, int Nq, int Nk, float sl2, cudaStream_t st) {
+  return causal ? launch_fwd<D, BF16, true>(mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st)
+                : launch_fwd<D, BF16, false>(mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st);
+}
+
+template <int D, bool BF16>
+attn_status dispatch_bwd_causal(int causal, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                const CUtensorMap& mdo, const void* o, const void* dout, const float* lse, void* dq,
+                                void* dk, void* dv, float* ws, int BH, int Nq, int Nk, float scale, int phase,
+                                cudaStream_t st) {
+  return causal
+             ? launch_bwd<D, BF16, true>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st)
+             : launch_bwd<D, BF16, false>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                     int d, float scale, int causal, attn_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_INVALID_ARG;
+  const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
+  if (cs != ATTN_OK) return cs;
+  const bool bf16 = dtype == ATTN_BF16;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, static_cast<long long>(BH) * Nq, d, bf16) ||
+      !make_map(&mk, k, static_cast<long long>(BH) * Nk, d, bf16) ||
+      !make_map(&mv, v, static_cast<long long>(BH) * Nk, d, bf16))
+    return ATTN_ERR_CUDA;
+  const float sl2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return bf16 ? dispatch_fwd_causal<64, true>(causal, mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st)
+                : dispatch_fwd_causal<64, false>(causal, mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st);
+  return bf16 ? dispatch_fwd_causal<128, true>(causal, mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st)
+              : dispatch_fwd_causal<128, false>(causal, mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return 0;
+  const unsigned long long rows = static_cast<unsigned long long>(B) * H * Nq;
+  const unsigned long long floats = rows * (static_cast<unsigned long long>(d) + 2);
+  if (floats > (~0ull) / 4) return 0;
+  return static_cast<size_t>(floats * 4);
+}
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
+                     int causal, attn_dtype dtype, void* stream) {
+  return attn_bwd_phase(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, causal, dtype,
+                        ATTN_BWD_ALL, stream);
+}
+
+attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                           const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq,
+                           int Nk, int d, float scale, int causal, attn_dtype dtype, int phase, void* stream) {
+  if (phase < ATTN_BWD_ALL || phase > ATTN_BWD_CONVERT) return ATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return ATTN_ERR_INVALID_ARG;
+  const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
+  if (cs != ATTN_OK) return cs;
+  const bool bf16 = dtype == ATTN_BF16;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, static_cast<long long>(BH) * Nq, d, bf16) ||
+      !make_map(&mk, k, static_cast<long long>(BH) * Nk, d, bf16) ||
+      !make_map(&mv, v, static_cast<long long>(BH) * Nk, d, bf16) ||
+      !make_map(&mdo, dout, static_cast<long long>(BH) * Nq, d, bf16))
+    return ATTN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  if (d == 64)
+    return bf16 ? dispatch_bwd_causal<64, true>(causal, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st)
+                : dispatch_bwd_causal<64, false>(causal, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st);
+  return bf16 ? dispatch_bwd_causal<128, true>(causal, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st)
+              : dispatch_bwd_causal<128, false>(causal, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st);
+}
+
+attn_status attn_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  int status = 0;
+  if (cudaMemcpyFromSymbol(&status, attn::g_device_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (status != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(attn::g_device_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return static_cast<attn_status>(status);
+}
+
+const char* attn_status_string(attn_status s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

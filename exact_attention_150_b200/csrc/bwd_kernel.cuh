@@ -1,0 +1,380 @@
+// bwd_kernel.cuh -- attention backward for sm_100a, by recomputation.
+//
+// The attention matrix is not stored by the forward pass; the backward pass
+// recomputes it from Q, K and the saved row log-sum-exp (page "FlashAttention
+// 核心原理", part 2 item 3).  Three kernels:
+//
+//   bwd_pre_kernel    D_i = sum_c dO_ic O_ic, -log2(e) * LSE_i, and dQacc = 0
+//   bwd_main_kernel   one CTA per (key tile j, batch*head): K_j, V_j stay in
+//                     shared memory; for every query tile i that sees them
+//                       S^T  = K_j Q_i^T              (tcgen05, TMEM)
+//                       dP^T = V_j dO_i^T             (tcgen05, TMEM)
+//                       P^T  = exp2(S^T * scale*log2e - LSE_i*log2e)
+//                       dS^T = P^T * (dP^T - D_i)
+//                       dV_j += P^T dO_i              (A = P^T from TMEM)
+//                       dK_j += dS^T Q_i              (A = dS^T from TMEM)
+//                       dQacc_i += scale * dS K_j     (fp32 atomics)
+//                     then dK_j = scale * dK_j and dV_j are written once.
+//   bwd_post_kernel   dQ = 16-bit(dQacc)
+//
+// Main-kernel CTA layout (384 threads):
+//   warp 0      TMA producer (K_j, V_j once; Q_i, dO_i through 2 stages)
+//   warp 1      MMA issuer (one thread)
+//   warp 2      TMEM allocation
+//   warps 4-7   P / dS computation, thread = key row = TMEM lane
+//   warps 8-11  dQ drain (thread = query row), then the dK/dV epilogue
+// Tensor memory: [0,128) S^T (P^T packed in [0,64)), [128,256) dP^T (dS^T
+// packed in [128,192)), [256,256+D) dV, [256+D,256+2D) dK, and the dQ tile in
+// the columns freed by packing: [64,128) and [192,256) (64 columns each).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+
+constexpr int kBwdTile = 128;
+
+template <int D>
+struct BwdLayout {
+  static constexpr int kChunkBytes = kBwdTile * 128;
+  static constexpr int kTileBytes = kBwdTile * D * 2;
+  static constexpr int kStages = 2;
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kTileBytes;
+  static constexpr int kStageOff = 2 * kTileBytes;  // stage s: Q at +s*2T, dO at +s*2T+T
+  static constexpr int kDSOff = kStageOff + kStages * 2 * kTileBytes;
+  static constexpr int kDSBytes = kBwdTile * kBwdTile * 2;
+  static constexpr int kBarOff = kDSOff + kDSBytes;
+  // kv_full, qd_full[S], qd_empty[S], s_full, dp_full, ds_full, dq_full, dq_free, acc_full, mma_done
+  static constexpr int kNumBars = 1 + 2 * kStages + 7;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+// One group of D/8 threads per row; each thread handles 8 elements.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256)
+    bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+                   const float* __restrict__ lse, float* __restrict__ dvec, float* __restrict__ nlse2,
+                   float* __restrict__ dqacc, long long rows) {
+  constexpr int kTpr = D / 8;
+  constexpr int kRowsPerBlock = 256 / kTpr;
+  const long long row = static_cast<long long>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kTpr;
+  const int seg = threadIdx.x % kTpr;
+  float acc = 0.f;
+  if (row < rows) {
+    const size_t off = static_cast<size_t>(row) * D + seg * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+    const uint4 b = *reinterpret_cast<const uint4*>(dout + off);
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = unpack2<BF16>(av[i]);
+      const float2 y = unpack2<BF16>(bv[i]);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
+    }
+    float4* z = reinterpret_cast<float4*>(dqacc + off);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int m = kTpr / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (row < rows && seg == 0) {
+    dvec[row] = acc;
+    nlse2[row] = -lse[row] * 1.4426950408889634074f;
+  }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256)
+    bwd_post_kernel(const float* __restrict__ dqacc, uint16_t* __restrict__ dq, long long n8) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(dqacc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(dqacc)[2 * i + 1];
+    reinterpret_cast<uint4*>(dq)[i] =
+        make_uint4(pack2<BF16>(a.x, a.y), pack2<BF16>(a.z, a.w), pack2<BF16>(b.x, b.y), pack2<BF16>(b.z, b.w));
+  }
+}
+
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const float* __restrict__ dvec, const float* __restrict__ nlse2, float* __restrict__ dqacc,
+                    uint16_t* __restrict__ dk_ptr, uint16_t* __restrict__ dv_ptr, int Nq, int Nk, float scale,
+                    float scale_log2) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* kv_full = bars;
+  uint64_t* qd_full = bars + 1;
+  uint64_t* qd_empty = qd_full + L::kStages;
+  uint64_t* s_full = qd_empty + L::kStages;
+  uint64_t* dp_full = s_full + 1;
+  uint64_t* ds_full = s_full + 2;
+  uint64_t* dq_full = s_full + 3;
+  uint64_t* dq_free = s_full + 4;
+  uint64_t* acc_full = s_full + 5;
+  uint64_t* mma_done = s_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int bh = blockIdx.x;
+  const int j = blockIdx.y;  // key tile; causal: small j has the most work and launches first
+  const int nqt = Nq / kBwdTile;
+  const int i0 = CAUSAL ? j : 0;
+  const int n_it = nqt - i0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&qd_full[s], 1);
+      mbar_init(&qd_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_full, 128);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      const int krow = bh * Nk + j * kBwdTile;
+      mbar_arrive_expect_tx(kv_full, 2 * L::kTileBytes);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_2d(smem + L::kKOff + c * L::kChunkBytes, &tm_k, kv_full, c * 64, krow);
+        tma_load_2d(smem + L::kVOff + c * L::kChunkBytes, &tm_v, kv_full, c * 64, krow);
+      }
+      int it = 0;
+      bool ok = true;
+      for (; it < n_it; ++it) {
+        const int s = it % L::kStages;
+        const uint32_t ph = (it / L::kStages) & 1;
+        if (!mbar_wait(&qd_empty[s], ph ^ 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int qrow = bh * Nq + (i0 + it) * kBwdTile;
+        mbar_arrive_expect_tx(&qd_full[s], 2 * L::kTileBytes);
+        uint8_t* qdst = smem + L::kStageOff + s * 2 * L::kTileBytes;
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_2d(qdst + c * L::kChunkBytes, &tm_q, &qd_full[s], c * 64, qrow);
+          tma_load_2d(qdst + L::kTileBytes + c * L::kChunkBytes, &tm_do, &qd_full[s], c * 64, qrow);
+        }
+      }
+      if (!ok) {
+        mbar_drain(kv_full, 0);
+        const int first = it > L::kStages ? it - L::kStages : 0;
+        for (int i = first; i < it; ++i) mbar_drain(&qd_full[i % L::kStages], (i / L::kStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);   // K-major x K-major
+      constexpr uint32_t kIdAcc = idesc_f16(BF16, 128, D, false, true);    // TMEM A x MN-major B
+      constexpr uint32_t kIdQ = idesc_f16(BF16, 128, 64, true, true);      // MN-major A x MN-major B
+      const uint32_t k_addr = smem_u32(smem + L::kKOff);
+      const uint32_t v_addr = smem_u32(smem + L::kVOff);
+      const uint32_t ds_addr = smem_u32(smem + L::kDSOff);
+      bool ok = mbar_wait(kv_full, 0, abort_flag);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it % L::kStages;
+        const uint32_t q_addr = smem_u32(smem + L::kStageOff + s * 2 * L::kTileBytes);
+        const uint32_t do_addr = q_addr + L::kTileBytes;
+        if (!mbar_wait(&qd_full[s], (it / L::kStages) & 1, abort_flag)) break;
+        // The dQ tile of the previous query tile occupies columns that S^T and
+        // dP^T overwrite: wait until it has been drained.
+        if (it > 0 && !mbar_wait(dq_free, (it - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
+          mma_ss(tmem + 0, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), kIdS,
+                 ks > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
+          mma_ss(tmem + 128, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024), kIdS,
+                 ks > 0 ? 1u : 0u);
+        }
+        mma_commit(dp_full);
+        if (!mbar_wait(ds_full, it & 1, abort_flag)) break;
+        tc_fence_after();
+        // dV += P^T dO and dK += dS^T Q: A from TMEM (8 columns per 16 queries),
+        // B MN-major with 16 query rows (2048 bytes) per K step.
+#pragma unroll
+        for (int ks = 0; ks < kBwdTile / 16; ++ks)
+          mma_ts(tmem + 256, tmem + 0 + ks * 8, sdesc_sw128(do_addr + ks * 2048, L::kChunkBytes, 1024), kIdAcc,
+                 (it > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < kBwdTile / 16; ++ks)
+          mma_ts(tmem + 256 + D, tmem + 128 + ks * 8, sdesc_sw128(q_addr + ks * 2048, L::kChunkBytes, 1024),
+                 kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&qd_empty[s]);
+        // dQ_i = dS K_j, in 64-column halves of the head dimension.
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+#pragma unroll
+          for (int ks = 0; ks < kBwdTile / 16; ++ks)
+            mma_ss(tmem + 64 + 128 * h, sdesc_sw128(ds_addr + ks * 2048, L::kChunkBytes, 1024),
+                   sdesc_sw128(k_addr + h * L::kChunkBytes + ks * 2048, L::kChunkBytes, 1024), kIdQ,
+                   ks > 0 ? 1u : 0u);
+        mma_commit(dq_full);
+        if (it == n_it - 1) mma_commit(acc_full);
+      }
+      mma_commit(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ P and dS
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // key row within tile j = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    uint8_t* ds_row = smem + L::kDSOff + r * 128;
+    for (int it = 0; it < n_it; ++it) {
+      const int i = i0 + it;
+      bool ok = mbar_wait(s_full, it & 1, abort_flag);
+      ok = ok && mbar_wait(dp_full, it & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const size_t vbase = static_cast<size_t>(bh) * Nq + static_cast<size_t>(i) * kBwdTile;
+      const float4* nl4 = reinterpret_cast<const float4*>(nlse2 + vbase);
+      const float4* dd4 = reinterpret_cast<const float4*>(dvec + vbase);
+#pragma unroll 1
+      for (int c = 0; c < kBwdTile / 16; ++c) {
+        uint32_t sr[16], pr[16];
+        tmem_ld16(tmem + lane_off + c * 16, sr);
+        tmem_ld16(tmem + lane_off + 128 + c * 16, pr);
+        float nl[16], dd[16];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float4 a = nl4[c * 4 + v];
+          const float4 b = dd4[c * 4 + v];
+          nl[4 * v] = a.x; nl[4 * v + 1] = a.y; nl[4 * v + 2] = a.z; nl[4 * v + 3] = a.w;
+          dd[4 * v] = b.x; dd[4 * v + 1] = b.y; dd[4 * v + 2] = b.z; dd[4 * v + 3] = b.w;
+        }
+        uint32_t ppk[8], dpk[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          float p0 = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, nl[e]));
+          float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), scale_log2, nl[e + 1]));
+          if (CAUSAL && i == j) {
+            // key r is visible to query q iff r <= q
+            if (r > c * 16 + e) p0 = 0.f;
+            if (r > c * 16 + e + 1) p1 = 0.f;
+          }
+          const float d0 = p0 * (__uint_as_float(pr[e]) - dd[e]);
+          const float d1 = p1 * (__uint_as_float(pr[e + 1]) - dd[e + 1]);
+          ppk[e / 2] = pack2<BF16>(p0, p1);
+          dpk[e / 2] = pack2<BF16>(d0, d1);
+        }
+        tmem_st8(tmem + lane_off + c * 8, ppk);
+        tmem_st8(tmem + lane_off + 128 + c * 8, dpk);
+        // dS^T row r, queries [16c, 16c+16): two 16-byte units of the
+        // 128-byte-swizzled MN-major tile (64 queries per 16 KB chunk).
+        uint8_t* chunk_row = ds_row + (c >> 2) * L::kChunkBytes;
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const int unit = ((c & 3) * 2 + v) ^ (r & 7);
+          *reinterpret_cast<uint4*>(chunk_row + unit * 16) =
+              make_uint4(dpk[4 * v], dpk[4 * v + 1], dpk[4 * v + 2], dpk[4 * v + 3]);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(ds_full);
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ dQ drain, dK/dV epilogue
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      ok = mbar_wait(dq_full, it & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      float* dst = dqacc + (static_cast<size_t>(bh) * Nq + static_cast<size_t>(i0 + it) * kBwdTile + row) * D;
+#pragma unroll 1
+      for (int h = 0; h < D / 64; ++h) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tmem + lane_off + 64 + 128 * h + 32 * c, rr);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            atomicAdd(reinterpret_cast<float4*>(dst + h * 64 + c * 32 + 4 * v),
+                      make_float4(__uint_as_float(rr[4 * v]) * scale, __uint_as_float(rr[4 * v + 1]) * scale,
+                                  __uint_as_float(rr[4 * v + 2]) * scale, __uint_as_float(rr[4 * v + 3]) * scale));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(dq_free);
+    }
+    if (ok && n_it > 0) {
+      ok = mbar_wait(acc_full, 0, abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        const size_t grow = static_cast<size_t>(bh) * Nk + static_cast<size_t>(j) * kBwdTile + row;
+        uint4* dvd = reinterpret_cast<uint4*>(dv_ptr + grow * D);
+        uint4* dkd = reinterpret_cast<uint4*>(dk_ptr + grow * D);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rv[32], pk[16];
+          tmem_ld32(tmem + lane_off + 256 + c * 32, rv);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack2<BF16>(__uint_as_float(rv[2 * e]), __uint_as_float(rv[2 * e + 1]));
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dvd[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          tmem_ld32(tmem + lane_off + 256 + D + c * 32, rv);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack2<BF16>(__uint_as_float(rv[2 * e]) * scale, __uint_as_float(rv[2 * e + 1]) * scale);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dkd[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,183 @@
+"""ctypes binding of libattn.so (include/attn.h).
+
+Argument marshalling only: the functions here turn torch tensors into device
+pointers, sizes and the current CUDA stream and call the C ABI; every step of
+the computation runs in the library's kernels.  If the library is missing or
+a call fails, they raise; there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libattn.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "attn.h")
+
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(5)
+ATTN_FP16, ATTN_BF16 = 0, 1
+ATTN_BWD_ALL, ATTN_BWD_PREPROCESS, ATTN_BWD_MAIN, ATTN_BWD_CONVERT = range(4)
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, where: str, status: int, message: str):
+        super().__init__(f"{where}: {message} (status {status})")
+        self.status = status
+
+
+def load() -> ctypes.CDLL:
+    """Loads libattn.so; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m exact_attention_150_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+    lib.attn_fwd.restype = st
+    lib.attn_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+    lib.attn_bwd.restype = st
+    lib.attn_bwd_phase.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
+    lib.attn_bwd_phase.restype = st
+    lib.attn_last_device_status.argtypes = [vp]
+    lib.attn_last_device_status.restype = st
+    lib.attn_status_string.argtypes = [st]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def declared_symbols() -> list[str]:
+    """Names of the functions include/attn.h declares."""
+    text = open(HEADER).read()
+    return re.findall(r"^\S.*?\b(attn_\w+)\s*\(", text, flags=re.M)
+
+
+def status_string(status: int) -> str:
+    return load().attn_status_string(status).decode()
+
+
+def _check(where: str, status: int) -> None:
+    if status != ATTN_OK:
+        raise AttnError(where, status, status_string(status))
+
+
+# ---------------------------------------------------------------- raw C ABI
+
+def attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
+    """Direct call of attn_fwd with integer device pointers; returns the status."""
+    return load().attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, int(causal), dtype, stream)
+
+
+def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
+    """Direct call of attn_bwd with integer device pointers; returns the status."""
+    return load().attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, int(causal),
+                           dtype, stream)
+
+
+def attn_bwd_phase(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, causal, dtype, phase,
+                   stream) -> int:
+    """Direct call of attn_bwd_phase (one of the three backward kernels)."""
+    return load().attn_bwd_phase(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale,
+                                 int(causal), dtype, phase, stream)
+
+
+def attn_bwd_workspace_bytes(B, H, Nq, Nk, d) -> int:
+    return int(load().attn_bwd_workspace_bytes(B, H, Nq, Nk, d))
+
+
+def attn_last_device_status(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return int(load().attn_last_device_status(stream))
+
+
+# ---------------------------------------------------------------- tensors
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return ATTN_FP16
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    raise TypeError(f"attention inputs must be float16 or bfloat16, got {t.dtype}")
+
+
+def _check_tensor(name: str, t: torch.Tensor, shape, dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None):
+    """O, LSE = attention(q, k, v) for q [B,H,Nq,d], k and v [B,H,Nk,d]."""
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    code = _dtype_code(q)
+    _check_tensor("q", q, (B, H, Nq, d), q.dtype)
+    _check_tensor("k", k, (B, H, Nk, d), q.dtype)
+    _check_tensor("v", v, (B, H, Nk, d), q.dtype)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check_tensor("out", out, (B, H, Nq, d), q.dtype)
+    _check_tensor("lse", lse, (B, H, Nq), torch.float32)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    _check("attn_fwd", attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                B, H, Nq, Nk, d, float(scale), causal, code, stream))
+    return out, lse
+
+
+def backward(q, k, v, out, lse, dout, causal: bool = False, scale: float | None = None,
+             dq=None, dk=None, dv=None, workspace=None, stream=None, phase: int = ATTN_BWD_ALL):
+    """dQ, dK, dV of attention for the output gradient dout.  `phase` runs
+    only one of the three backward kernels (see attn_bwd_phase)."""
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    code = _dtype_code(q)
+    for name, t, shp in (("q", q, (B, H, Nq, d)), ("k", k, (B, H, Nk, d)), ("v", v, (B, H, Nk, d)),
+                         ("out", out, (B, H, Nq, d)), ("dout", dout, (B, H, Nq, d))):
+        _check_tensor(name, t, shp, q.dtype)
+    _check_tensor("lse", lse, (B, H, Nq), torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        _check_tensor(name, t, ref.shape, q.dtype)
+    nbytes = attn_bwd_workspace_bytes(B, H, Nq, Nk, d)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    if workspace.numel() * workspace.element_size() < nbytes or not workspace.is_cuda:
+        raise ValueError(f"workspace must be a CUDA buffer of at least {nbytes} bytes")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    _check("attn_bwd", attn_bwd_phase(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                      workspace.data_ptr(), B, H, Nq, Nk, d, float(scale), causal, code, phase,
+                                      stream))
+    return dq, dk, dv
+
+
+def device_status(stream=None) -> None:
+    """Raises if a kernel of the library recorded an error (e.g. a wait timeout)."""
+    _check("attn_last_device_status", attn_last_device_status(stream))

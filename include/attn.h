@@ -1,0 +1,146 @@
+/*
+ * attn.h -- C ABI of libattn.so: exact scaled-dot-product attention on one
+ * B200 (sm_100a), forward and backward.
+ *
+ * The operation is the one defined on the page "FlashAttention 核心原理"
+ * (cxbdf.cn), part 1: Attention(Q, K, V) = softmax(Q K^T * scale) V, with an
+ * optional causal mask.  It is computed tile by tile with an online softmax
+ * (same page, part 2: tiling and kernel fusion), so the Nq x Nk score matrix is
+ * never written to device memory.  The backward pass recomputes the attention
+ * probabilities from the saved per-row log-sum-exp instead of storing them
+ * (same page, part 2 item 3, "recomputation for the backward pass").  The
+ * argument list follows the forward kernel interface sketched on the page
+ * "FlashAttention-2 性能革命", section 2.1 (q, k, v, o, softmax_lse, seqlen_q,
+ * seqlen_k, num_heads, softmax_scale) and the user call
+ * flash_attn_func(q, k, v, softmax_scale, causal) of the same page, section 3.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.  Q, O, dO, dQ are contiguous [B][H][Nq][d]; K, V, dK, dV are
+ *   contiguous [B][H][Nk][d]; LSE is contiguous [B][H][Nq] float.  Element
+ *   type is fp16 or bf16 (attn_dtype) for every 16-bit tensor of one call.
+ * Memory.  Every pointer is a DEVICE pointer on the current CUDA device,
+ *   16-byte aligned, allocated and owned by the caller.  The library keeps no
+ *   allocation of its own between calls.
+ * Stream.  `stream` is a cudaStream_t (NULL = legacy default stream).  Every
+ *   call only enqueues work on it and returns without synchronising.
+ * Mask.  causal != 0 applies the top-left causal mask: query row i attends to
+ *   key row j iff j <= i.  (The pages name a causal mask but not its
+ *   alignment when Nq != Nk; top-left is the reading taken.)
+ * LSE.  lse[b][h][i] = ln sum_j exp(scale * q_i . k_j) over the unmasked j:
+ *   the natural-log row log-sum-exp of the scaled scores, in fp32.
+ * Supported shapes.  d in {64, 128}; Nq and Nk multiples of 128; for causal,
+ *   Nq == Nk.  Other shapes return ATTN_ERR_UNSUPPORTED.
+ * Errors.  Arguments are validated on the host before anything is enqueued:
+ *   a NULL pointer, a non-positive size or a pointer that is not 16-byte
+ *   aligned returns ATTN_ERR_INVALID_ARG; an unsupported shape or dtype returns
+ *   ATTN_ERR_UNSUPPORTED; a failed launch returns ATTN_ERR_CUDA.  Nothing is
+ *   written to any output when a call returns an error.  There is no fallback
+ *   to another implementation.  Kernels never trap: a wait inside a kernel
+ *   that exceeds its time limit makes the kernel record ATTN_ERR_TIMEOUT in a
+ *   device status word and return early; attn_last_device_status() reads it.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,
+  ATTN_ERR_UNSUPPORTED = 2,
+  ATTN_ERR_CUDA = 3,
+  ATTN_ERR_TIMEOUT = 4
+} attn_status;
+
+typedef enum { ATTN_FP16 = 0, ATTN_BF16 = 1 } attn_dtype;
+
+/*
+ * Forward pass.  Writes O = softmax(scale * Q K^T [+ causal mask]) V (16-bit,
+ * round to nearest even) and LSE (fp32, see above).  The probabilities P are
+ * rounded to the 16-bit input type before the product with V; all sums
+ * accumulate in fp32.
+ *   q, k, v   inputs, read only.
+ *   o         output [B][H][Nq][d], 16-bit.
+ *   lse       output [B][H][Nq], float.
+ *   B, H      batch and head count (> 0).
+ *   Nq, Nk    query and key sequence lengths (> 0).
+ *   d         head dimension.
+ *   scale     multiplier of Q K^T; the pages use 1/sqrt(d).
+ */
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                     attn_dtype dtype, void* stream);
+
+/*
+ * Size in bytes of the device workspace attn_bwd needs: an fp32 dQ
+ * accumulator [B][H][Nq][d], then the fp32 row term D [B][H][Nq], then the
+ * fp32 row term -log2(e) * LSE [B][H][Nq].  Returns 0 if a size is
+ * non-positive or the total overflows size_t.
+ */
+size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d);
+
+/*
+ * Backward pass of attn_fwd for the loss gradient dO.  Recomputes P from
+ * (q, k, lse) and writes
+ *   dV = P^T dO,  dS = P * (dO V^T - D),  dQ = scale * dS K,  dK = scale * dS^T Q,
+ * where D_i = sum_c dO_ic O_ic.  `o` and `lse` must be the outputs of attn_fwd
+ * for the same q, k, v, scale and causal flag.
+ *   dq, dk, dv   outputs, 16-bit, same layouts as q, k, v.
+ *   workspace    device buffer of attn_bwd_workspace_bytes() bytes, 16-byte
+ *                aligned; its contents on entry are ignored and on return are
+ *                unspecified.  It must not be shared by calls that overlap.
+ * dQ is accumulated with fp32 atomic additions, so its last bits may differ
+ * between runs; dK and dV are deterministic.
+ */
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                     void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
+                     int causal, attn_dtype dtype, void* stream);
+
+/*
+ * One phase of attn_bwd, for callers that time or schedule the three
+ * backward kernels separately.  Running ATTN_BWD_PREPROCESS, ATTN_BWD_MAIN
+ * and ATTN_BWD_CONVERT in that order on one stream, with the same arguments
+ * and workspace, is exactly attn_bwd; ATTN_BWD_ALL is attn_bwd itself.
+ *   PREPROCESS  D_i = sum_c dO_ic O_ic and -log2(e) LSE_i into the workspace,
+ *               and zeroes the dQ accumulator;
+ *   MAIN        recomputes P and accumulates dV, dK (written to dv, dk) and
+ *               the fp32 dQ accumulator;
+ *   CONVERT     dq = 16-bit(dQ accumulator).
+ * Arguments, validation and errors as for attn_bwd; `phase` outside the
+ * enum returns ATTN_ERR_INVALID_ARG.
+ */
+typedef enum {
+  ATTN_BWD_ALL = 0,
+  ATTN_BWD_PREPROCESS = 1,
+  ATTN_BWD_MAIN = 2,
+  ATTN_BWD_CONVERT = 3
+} attn_bwd_phase_t;
+
+attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                           void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
+                           int causal, attn_dtype dtype, int phase, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word that
+ * kernels of this library set when a bounded wait times out
+ * (ATTN_ERR_TIMEOUT), or ATTN_ERR_CUDA if the synchronisation itself fails.
+ * ATTN_OK means no kernel of this library has recorded an error since the
+ * previous call on this device.
+ */
+attn_status attn_last_device_status(void* stream);
+
+/* A static, human-readable name for a status code (never NULL). */
+const char* attn_status_string(attn_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

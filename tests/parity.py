@@ -1,0 +1,84 @@
+"""Shared helpers of the GPU parity tests: exact upcasts, per-slice oracle
+calls and the tolerance checks.
+
+Tolerances (attention parity bar for this library):
+  O:   max |O_gpu - O_ref| <= 2e-3 (fp16) or 1e-2 (bf16);
+  LSE: max |LSE_gpu - LSE_ref| <= 1e-3;
+  dQ, dK, dV: ||G_gpu - G_ref||_F / ||G_ref||_F <= 2e-2.
+O is stored in 16 bits, and half a unit in the last place of a 16-bit
+number exceeds the O tolerance once |O| >= 4 (bf16) or >= 8 (fp16).  Those
+elements are checked against one unit in the last place of the 16-bit type
+at |O_ref| instead; every other element is held to the stated tolerance.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+O_TOL = {torch.float16: 2e-3, torch.bfloat16: 1e-2}
+LSE_TOL = 1e-3
+GRAD_TOL = 2e-2
+_MANT = {torch.float16: 10, torch.bfloat16: 7}
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    """Exact upcast of a (16-bit or fp32) tensor to a float64 array."""
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def ulp16(x: np.ndarray, dtype: torch.dtype) -> np.ndarray:
+    e = np.floor(np.log2(np.maximum(np.abs(x), 1e-30)))
+    return np.exp2(e - _MANT[dtype])
+
+
+def o_violations(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype) -> tuple[int, float]:
+    """Number of O elements outside the bar, and the max abs error."""
+    err = np.abs(got - ref)
+    allow = np.where(0.5 * ulp16(ref, dtype) > O_TOL[dtype], ulp16(ref, dtype), O_TOL[dtype])
+    return int(np.count_nonzero(err > allow)), float(err.max(initial=0.0))
+
+
+def rel_fro(got: np.ndarray, ref: np.ndarray) -> float:
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
+
+
+def assert_o(got, ref, dtype, what=""):
+    n, mx = o_violations(got, ref, dtype)
+    assert n == 0, f"{what}: {n} O elements outside tolerance (max abs err {mx:.3e})"
+
+
+def assert_lse(got, ref, what=""):
+    err = float(np.max(np.abs(got - ref), initial=0.0))
+    assert err <= LSE_TOL, f"{what}: LSE max abs err {err:.3e}"
+
+
+def assert_grad(got, ref, name, what=""):
+    e = rel_fro(got, ref)
+    assert e <= GRAD_TOL, f"{what}: {name} relative Frobenius error {e:.3e}"
+
+
+def oracle_forward_slices(q, k, v, scale, causal, slices, rows=None):
+    """Oracle O and LSE for the given flat (b*h) slices, optionally only for
+    query rows `rows` (absolute indices, ascending)."""
+    B, H, Nq, d = q.shape
+    qf, kf, vf = (t.reshape(B * H, t.shape[2], d) for t in (q, k, v))
+    outs, lses = [], []
+    for s in slices:
+        k64, v64 = f64(kf[s]), f64(vf[s])
+        if rows is None:
+            o, lse, _ = oracle.forward(f64(qf[s]), k64, v64, scale, causal)
+        else:
+            o = np.empty((len(rows), d))
+            lse = np.empty(len(rows))
+            q64 = f64(qf[s])
+            for r in rows:  # one row at a time: the oracle sees exactly that query
+                oo, ll, _ = oracle.forward(q64[r:r + 1], k64, v64, scale, causal, q_offset=r)
+                i = rows.index(r)
+                o[i], lse[i] = oo[0], ll[0]
+        outs.append(o)
+        lses.append(lse)
+    return outs, lses

@@ -1,0 +1,131 @@
+"""The C ABI library on the host (no GPU): it loads, exports every symbol that
+include/attn.h declares, and rejects bad arguments before touching CUDA."""
+
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from exact_attention_150_b200 import build, native
+
+FAKE = 0x10000  # 16-byte aligned; never dereferenced: every case below fails validation first
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return native.load()
+
+
+def test_header_declares_the_boundary():
+    names = set(native.declared_symbols())
+    assert {"attn_fwd", "attn_bwd", "attn_bwd_phase", "attn_bwd_workspace_bytes", "attn_last_device_status",
+            "attn_status_string"} <= names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in native.declared_symbols():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", native.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = {line.split()[-1] for line in out.stdout.splitlines() if line.strip()}
+    for name in native.declared_symbols():
+        assert name in exported, name
+
+
+def test_library_is_built_for_sm100a(lib):
+    out = subprocess.run(["cuobjdump", "--list-elf", native.LIB_PATH], capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    assert "sm_100a" in out.stdout
+
+
+def test_status_strings(lib):
+    assert native.status_string(0) == "ok"
+    for s in range(1, 5):
+        assert native.status_string(s) not in ("ok", "")
+    assert native.status_string(99) == "unknown status"
+
+
+def _fwd(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, H=1, Nq=128, Nk=128, d=64, scale=0.125, causal=0,
+                dtype=native.ATTN_BF16, stream=None)
+    args.update(kw)
+    return native.attn_fwd(**args)
+
+
+def _bwd(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, workspace=FAKE,
+                B=1, H=1, Nq=128, Nk=128, d=64, scale=0.125, causal=0, dtype=native.ATTN_FP16, stream=None)
+    args.update(kw)
+    return native.attn_bwd(**args)
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "o", "lse"])
+def test_fwd_null_pointer(lib, field):
+    assert _fwd(**{field: None}) == native.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "o", "lse", "dout", "dq", "dk", "dv", "workspace"])
+def test_bwd_null_and_misaligned_pointer(lib, field):
+    assert _bwd(**{field: None}) == native.ATTN_ERR_INVALID_ARG
+    assert _bwd(**{field: FAKE + 8}) == native.ATTN_ERR_INVALID_ARG
+
+
+def test_fwd_misaligned_pointer(lib):
+    assert _fwd(q=FAKE + 2) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd(lse=FAKE + 4) == native.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("field", ["B", "H", "Nq", "Nk", "d"])
+@pytest.mark.parametrize("value", [0, -128])
+def test_non_positive_sizes(lib, field, value):
+    assert _fwd(**{field: value}) == native.ATTN_ERR_INVALID_ARG
+    assert _bwd(**{field: value}) == native.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(d=96), dict(d=256), dict(d=32), dict(Nq=200), dict(Nk=130),
+                                dict(Nq=128, Nk=256, causal=1), dict(dtype=2), dict(dtype=-1)])
+def test_unsupported_shapes(lib, kw):
+    assert _fwd(**kw) == native.ATTN_ERR_UNSUPPORTED
+    assert _bwd(**kw) == native.ATTN_ERR_UNSUPPORTED
+
+
+def test_workspace_size(lib):
+    assert native.attn_bwd_workspace_bytes(2, 16, 4096, 4096, 64) == 4 * 2 * 16 * 4096 * (64 + 2)
+    assert native.attn_bwd_workspace_bytes(1, 16, 16384, 16384, 128) == 4 * 16 * 16384 * 130
+    assert native.attn_bwd_workspace_bytes(0, 1, 128, 128, 64) == 0
+    assert native.attn_bwd_workspace_bytes(1, 1, -1, 128, 64) == 0
+
+
+def test_tensor_wrapper_rejects_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        native.forward(q, q, q)
+    with pytest.raises(TypeError):
+        native.forward(q.float(), q.float(), q.float())
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(native, "_lib", None)
+    monkeypatch.setattr(native, "LIB_PATH", str(tmp_path / "libattn.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        native.load()
+
+
+@pytest.mark.parametrize("phase", [-1, 4, 99])
+def test_bwd_phase_out_of_range(lib, phase):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, workspace=FAKE,
+                B=1, H=1, Nq=128, Nk=128, d=64, scale=0.125, causal=0, dtype=native.ATTN_FP16, phase=phase,
+                stream=None)
+    assert native.attn_bwd_phase(**args) == native.ATTN_ERR_INVALID_ARG
+
+
+def test_bwd_phase_validates_like_bwd(lib):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, workspace=FAKE,
+                B=1, H=1, Nq=128, Nk=128, d=96, scale=0.125, causal=0, dtype=native.ATTN_FP16,
+                phase=native.ATTN_BWD_MAIN, stream=None)
+    assert native.attn_bwd_phase(**args) == native.ATTN_ERR_UNSUPPORTED
+    args.update(d=64, dq=None)
+    assert native.attn_bwd_phase(**args) == native.ATTN_ERR_INVALID_ARG

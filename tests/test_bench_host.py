@@ -1,0 +1,79 @@
+"""Host-side logic of bench.py (no GPU): the max-over-ranks timing and the
+whole-job aggregation on two gloo ranks, the clock-sample parser, and the
+reference arm (the fp64 oracle on the host cores) on a small sequence."""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    local_ms = 100.0 + 50.0 * rank  # rank 1 is the slow one
+    m = bench.max_over_ranks(local_ms, world)
+    out[rank] = (m, bench.aggregate(1e12, 10, world, m))
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_aggregate_two_gloo_ranks():
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    port = 29500 + os.getpid() % 1000
+    mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
+    for r in range(world):
+        m, v = out[r]
+        assert m == 150.0
+        # 2 ranks x 10 steps x 1 TFLOP in 150 ms
+        assert v == pytest.approx(2 * 10 * 1e12 / 0.150 / 1e12)
+
+
+def test_single_rank_is_identity():
+    assert bench.max_over_ranks(12.5, 1) == 12.5
+    assert bench.aggregate(2e12, 5, 1, 1000.0) == pytest.approx(10.0)
+
+
+def test_clock_sample_parser():
+    c = bench.ClockSampler(0)
+    c.lines = ["0, 1800, 1965, 900.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+               "0, 1700, 1965, 950.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+               "0, 1900, 1965, 500.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active"]
+    s = c.summary()
+    assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"]
+
+
+def test_sample_flops_counts_visible_keys():
+    from exact_attention_150_b200 import workloads
+    w = workloads.LONG_CTX
+    # causal: row r sees r+1 keys; 4 d flops per key forward, 3.5x with backward
+    assert bench.sample_flops(w, [0, 9]) == 4.0 * w.d * (1 + 10) * 3.5
+
+
+def test_reference_arm_prints_one_line():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--seq", "1024",
+                          "--steps", "2", "--warmup", "1"], capture_output=True, text=True, env=env, timeout=600)
+    assert out.returncode == 0, out.stderr
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "TFLOP/s"
+    assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["higher_is_better"] is True
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--seq", "256",
+                          "--steps", "1", "--warmup", "0"], capture_output=True, text=True, env=env, timeout=300)
+    assert out.returncode == 0 and out.stdout.strip() == ""

@@ -1,0 +1,117 @@
+"""Backward parity: dQ, dK, dV from the CUDA library (forward then backward,
+through the C ABI) against the fp64 oracle's gradients of the same inputs.
+
+The GPU backward uses the GPU forward's O and LSE, as a training step would;
+the oracle differentiates the exact definition.  Small shapes are checked in
+full; the long-context workload is checked where the oracle's answer is exact
+on a window (query rows [0, 1024) and key rows [N-1024, N) under the causal
+mask) and through the gradient identities over the whole run.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_attention_150_b200 import native, workloads
+from exact_attention_150_b200.workloads import draw
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def run_fwd_bwd(q, k, v, do, causal, scale):
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = native.forward(qd, kd, vd, causal=causal, scale=scale)
+    dq, dk, dv = native.backward(qd, kd, vd, o, lse, dod, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    native.device_status()
+    return o.cpu(), lse.cpu(), dq.cpu(), dk.cpu(), dv.cpu()
+
+
+def check_grads_all_slices(q, k, v, do, causal, scale, what):
+    o, lse, dq, dk, dv = run_fwd_bwd(q, k, v, do, causal, scale)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    flat = lambda t, n: t.reshape(B * H, n, d)
+    for s in range(B * H):
+        args = [parity.f64(flat(t, n)[s]) for t, n in ((q, Nq), (k, Nk), (v, Nk), (do, Nq))]
+        ro, rlse, _ = oracle.forward(*args[:3], scale, causal)
+        rdq, rdk, rdv = oracle.backward(*args, scale, causal)
+        tag = f"{what} slice {s}"
+        parity.assert_o(parity.f64(flat(o, Nq)[s]), ro, q.dtype, tag)
+        parity.assert_lse(parity.f64(lse.reshape(B * H, Nq)[s]), rlse, tag)
+        parity.assert_grad(parity.f64(flat(dq, Nq)[s]), rdq, "dQ", tag)
+        parity.assert_grad(parity.f64(flat(dk, Nk)[s]), rdk, "dK", tag)
+        parity.assert_grad(parity.f64(flat(dv, Nk)[s]), rdv, "dV", tag)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n", [128, 384, 640])
+def test_backward_small(dtype, d, causal, n):
+    q, k, v, do = draw(1, 2, n, n, d, dtype, seed=200 + n + d, with_grad=True)
+    check_grads_all_slices(q, k, v, do, causal, 1.0 / math.sqrt(d), f"N{n} d{d} {dtype} causal={causal}")
+
+
+@pytest.mark.parametrize("nq,nk", [(256, 512), (512, 256)])
+def test_backward_nq_ne_nk(nq, nk):
+    q, k, v, do = draw(1, 2, nq, nk, 64, torch.float16, seed=21, with_grad=True)
+    check_grads_all_slices(q, k, v, do, False, 0.125, f"Nq{nq} Nk{nk}")
+
+
+def test_backward_scale_zero_gives_zero_dq_dk():
+    q, k, v, do = draw(1, 2, 256, 256, 64, torch.bfloat16, seed=22, with_grad=True)
+    _, _, dq, dk, dv = run_fwd_bwd(q, k, v, do, True, 0.0)
+    assert torch.count_nonzero(dq) == 0 and torch.count_nonzero(dk) == 0
+    check_grads_all_slices(q, k, v, do, True, 0.0, "scale 0")
+
+
+def test_backward_repeatable_dk_dv():
+    """dK and dV involve no atomics: two runs give identical bits."""
+    q, k, v, do = draw(1, 4, 512, 512, 128, torch.bfloat16, seed=23, with_grad=True)
+    a = run_fwd_bwd(q, k, v, do, True, 1 / math.sqrt(128))
+    b = run_fwd_bwd(q, k, v, do, True, 1 / math.sqrt(128))
+    assert torch.equal(a[3], b[3]) and torch.equal(a[4], b[4])
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_train_d64_workload_all_slices():
+    w = workloads.TRAIN_D64
+    q, k, v, do = workloads.make_inputs(w)
+    check_grads_all_slices(q, k, v, do, w.causal, w.scale, w.label())
+
+
+def test_long_context_workload_windows_and_identities():
+    w = workloads.LONG_CTX
+    q, k, v, do = workloads.make_inputs(w)
+    o, lse, dq, dk, dv = run_fwd_bwd(q, k, v, do, w.causal, w.scale)
+    n, win, d = w.N, 1024, w.d
+    qf, kf, vf, dof = (t.reshape(w.B * w.H, n, d) for t in (q, k, v, do))
+    of, lf, dqf, dkf, dvf = (t.reshape(w.B * w.H, n, -1) if t.dim() == 4 else t.reshape(w.B * w.H, n)
+                             for t in (o, lse, dq, dk, dv))
+    for s in range(w.B * w.H):
+        tag = f"{w.label()} head {s}"
+        # Query rows [0, win) see only keys [0, win): the prefix sub-problem is exact.
+        pq, pk, pv, pdo = (parity.f64(t[s, :win]) for t in (qf, kf, vf, dof))
+        ro, rl, _ = oracle.forward(pq, pk, pv, w.scale, True)
+        parity.assert_o(parity.f64(of[s, :win]), ro, q.dtype, tag + " rows<1024")
+        parity.assert_lse(parity.f64(lf[s, :win]), rl, tag + " rows<1024")
+        if s < 4:
+            rdq, _, _ = oracle.backward(pq, pk, pv, pdo, w.scale, True)
+            parity.assert_grad(parity.f64(dqf[s, :win]), rdq, "dQ rows<1024", tag)
+            # Key rows [n-win, n) receive gradient only from query rows [n-win, n).
+            sq, sdo = parity.f64(qf[s, n - win:]), parity.f64(dof[s, n - win:])
+            _, rdk, rdv = oracle.backward(sq, parity.f64(kf[s]), parity.f64(vf[s]), sdo, w.scale, True,
+                                          q_offset=n - win)
+            parity.assert_grad(parity.f64(dkf[s, n - win:]), rdk[n - win:], "dK keys>=N-1024", tag)
+            parity.assert_grad(parity.f64(dvf[s, n - win:]), rdv[n - win:], "dV keys>=N-1024", tag)
+        # Whole run: sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i.
+        gk, gv, gdo = parity.f64(dkf[s]), parity.f64(dvf[s]), parity.f64(dof[s])
+        assert np.linalg.norm(gk.sum(0)) <= parity.GRAD_TOL * np.linalg.norm(gk), tag + " sum dK"
+        assert np.linalg.norm(gv.sum(0) - gdo.sum(0)) <= parity.GRAD_TOL * np.linalg.norm(gv), tag + " sum dV"

@@ -1,0 +1,138 @@
+"""Forward parity: the CUDA library (through the C ABI) against the fp64 oracle,
+element by element, on seeded inputs.
+
+Small shapes span several tiles, an odd number of query tiles (a CTA with a
+single tile) and Nq != Nk.  The named workloads run at full size: every slice
+of the tiny, 7B-layer and short sweep workloads, and sampled slices and rows
+of the long sweep points and of the long-context workload.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_attention_150_b200 import native, workloads
+from exact_attention_150_b200.workloads import draw
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def run_forward(q, k, v, causal, scale):
+    qd, kd, vd = (t.to(DEV) for t in (q, k, v))
+    o, lse = native.forward(qd, kd, vd, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    native.device_status()
+    return o.cpu(), lse.cpu()
+
+
+def check_all_slices(q, k, v, causal, scale, what):
+    o, lse = run_forward(q, k, v, causal, scale)
+    B, H, Nq, d = q.shape
+    refs, lrefs = parity.oracle_forward_slices(q, k, v, scale, causal, range(B * H))
+    of, lf = o.reshape(B * H, Nq, d), lse.reshape(B * H, Nq)
+    for s in range(B * H):
+        parity.assert_o(parity.f64(of[s]), refs[s], q.dtype, f"{what} slice {s}")
+        parity.assert_lse(parity.f64(lf[s]), lrefs[s], f"{what} slice {s}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n", [128, 256, 640])
+def test_forward_small(dtype, d, causal, n):
+    q, k, v = draw(2, 3, n, n, d, dtype, seed=100 + n + d)
+    check_all_slices(q, k, v, causal, 1.0 / math.sqrt(d), f"N{n} d{d} {dtype} causal={causal}")
+
+
+@pytest.mark.parametrize("nq,nk", [(384, 768), (768, 256), (128, 1024)])
+def test_forward_nq_ne_nk(nq, nk):
+    q, k, v = draw(1, 2, nq, nk, 128, torch.bfloat16, seed=7)
+    check_all_slices(q, k, v, False, 1.0 / math.sqrt(128), f"Nq{nq} Nk{nk}")
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.3, 0.9])
+def test_forward_other_scales(scale):
+    q, k, v = draw(1, 2, 256, 256, 64, torch.float16, seed=9)
+    for causal in (False, True):
+        check_all_slices(q, k, v, causal, scale, f"scale {scale} causal={causal}")
+
+
+def test_forward_large_scores_need_rescaling():
+    """Scores growing along the key axis force the running maximum to move by
+    far more than the lazy-rescale threshold on every tile."""
+    d = 64
+    q, k, v = draw(1, 1, 512, 512, d, torch.bfloat16, seed=11)
+    ramp = torch.linspace(0, 6, 512).reshape(1, 1, 512, 1)
+    k = (k.float() * 0.2 + ramp).to(torch.bfloat16)
+    q = torch.full_like(q, 1.0)
+    check_all_slices(q, k, v, False, 1.0, "ramp non-causal")
+    check_all_slices(q, k, v, True, 1.0, "ramp causal")
+
+
+def test_forward_constant_v_and_first_causal_row():
+    q, k, v = draw(1, 4, 256, 256, 128, torch.bfloat16, seed=12)
+    vc = v[:, :, :1, :].expand_as(v).contiguous()
+    o, _ = run_forward(q, k, vc, True, 1 / math.sqrt(128))
+    parity.assert_o(parity.f64(o), parity.f64(vc), q.dtype, "constant V")
+    o, lse = run_forward(q, k, v, True, 1 / math.sqrt(128))
+    assert torch.equal(o[:, :, 0], v[:, :, 0])
+    want = (q[:, :, 0].double() * k[:, :, 0].double()).sum(-1) / math.sqrt(128)
+    np.testing.assert_allclose(lse[:, :, 0].double().numpy(), want.numpy(), atol=1e-4)
+
+
+def test_forward_unsupported_shapes_raise():
+    q = torch.zeros(1, 1, 200, 64, dtype=torch.float16, device=DEV)
+    with pytest.raises(native.AttnError):
+        native.forward(q, q, q)
+    q = torch.zeros(1, 1, 128, 96, dtype=torch.float16, device=DEV)
+    with pytest.raises(native.AttnError):
+        native.forward(q, q, q)
+
+
+# ---------------------------------------------------------- named workloads
+
+def test_tiny_workload():
+    w = workloads.TINY
+    q, k, v = workloads.make_inputs(w, with_grad=False)
+    check_all_slices(q, k, v, w.causal, w.scale, w.label())
+
+
+def test_layer7b_workload_all_slices():
+    w = workloads.LAYER_7B
+    q, k, v = workloads.make_inputs(w, with_grad=False)
+    check_all_slices(q, k, v, w.causal, w.scale, w.label())
+
+
+@pytest.mark.parametrize("n", [512, 1024, 2048])
+def test_sweep_workload_all_slices(n):
+    w = workloads.SWEEP[n]
+    q, k, v = workloads.make_inputs(w, with_grad=False)
+    check_all_slices(q, k, v, w.causal, w.scale, w.label())
+
+
+def _sampled_rows(n, count, seed):
+    r = np.random.default_rng(seed)
+    rows = {0, 1, 127, 128, n - 129, n - 128, n - 1}
+    rows.update(int(x) for x in r.choice(n, size=count, replace=False))
+    return sorted(x for x in rows if 0 <= x < n)
+
+
+@pytest.mark.parametrize("n", [4096, 8192])
+def test_sweep_workload_sampled(n):
+    w = workloads.SWEEP[n]
+    q, k, v = workloads.make_inputs(w, with_grad=False)
+    o, lse = run_forward(q, k, v, w.causal, w.scale)
+    B, H = w.B, w.H
+    slices = [0, 37, B * H - 1]
+    rows = _sampled_rows(n, 48, n)
+    refs, lrefs = parity.oracle_forward_slices(q, k, v, w.scale, w.causal, slices, rows)
+    of, lf = o.reshape(B * H, n, w.d), lse.reshape(B * H, n)
+    for s, ref, lref in zip(slices, refs, lrefs):
+        parity.assert_o(parity.f64(of[s][rows]), ref, q.dtype, f"{w.label()} slice {s}")
+        parity.assert_lse(parity.f64(lf[s][rows]), lref, f"{w.label()} slice {s}")
