@@ -239,31 +239,45 @@ __global__ void __launch_bounds__(384, 1)
     const int qt = 2 * pair + t;
     float m_run = -INFINITY;  // running max of the scores, log2 units (stale by < 8)
     float l_run = 0.f;        // running sum of exp2(score - m_run)
+    float l_o = 0.f;          // the same sum over the 16-bit rounded terms
+    const bool pos_scale = scale_log2 > 0.f;
+    const float cx = pos_scale ? scale_log2 : 1.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       ok = mbar_wait(&s_full[t], j & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      // Scores of this row.  With a positive scale, the scale is folded into
+      // the exponent's FMA and the maximum is taken on the raw scores;
+      // otherwise the scores are scaled first.
       float x[kTile];
 #pragma unroll
       for (int c = 0; c < kTile / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(s_tm + c * 32, r);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]) * scale_log2;
+        for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
+      }
+      if (!pos_scale) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) x[c] *= scale_log2;
       }
       if (CAUSAL && j == qt) {
 #pragma unroll
         for (int c = 0; c < kTile; ++c)
           if (c > row) x[c] = -INFINITY;
       }
-      float mx = x[0];
+      float mp[8];
 #pragma unroll
-      for (int c = 1; c < kTile; ++c) mx = fmaxf(mx, x[c]);
-      const float m_new = fmaxf(m_run, mx);
-      // Rescale O and l only when the maximum has grown by more than 2^8;
-      // otherwise keep the stale maximum (P stays below 256).
+      for (int i = 0; i < 8; ++i) mp[i] = x[i];
+#pragma unroll
+      for (int c = 8; c < kTile; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+      const float m_tile = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                 fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * cx;
+      const float m_new = fmaxf(m_run, m_tile);
+      // Rescale O and the sums only when the maximum has grown by more than
+      // 2^8; otherwise keep the stale maximum (P stays below 256).
       const bool need = (j > 0) && (m_new - m_run > 8.f);
       if (j == 0) m_run = m_new;
       if (__any_sync(0xffffffffu, need)) {
@@ -278,26 +292,31 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (need) {
           l_run *= alpha;
+          l_o *= alpha;
           m_run = m_new;
         }
       }
-      float rs = 0.f;
+      // l_run sums the fp32 probabilities (for LSE); l_o sums the rounded
+      // 16-bit probabilities that the P V product uses, so that O / l_o is a
+      // weighted mean of V rows with weights summing to one.
+      float su[4] = {0.f, 0.f, 0.f, 0.f}, sr[4] = {0.f, 0.f, 0.f, 0.f};
+      const float neg_m = -m_run;
 #pragma unroll
       for (int c = 0; c < kTile / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(x[c * 32 + 2 * i] - m_run);
-          const float p1 = ex2(x[c * 32 + 2 * i + 1] - m_run);
+          const float p0 = ex2(fmaf(x[c * 32 + 2 * i], cx, neg_m));
+          const float p1 = ex2(fmaf(x[c * 32 + 2 * i + 1], cx, neg_m));
           pk[i] = pack2<BF16>(p0, p1);
-          // Sum the rounded probabilities that the P V product uses, so that
-          // O is a weighted mean of V rows with weights summing to one.
           const float2 pr = unpack2<BF16>(pk[i]);
-          rs += pr.x + pr.y;
+          su[i & 3] += p0 + p1;
+          sr[i & 3] += pr.x + pr.y;
         }
         tmem_st16(s_tm + c * 16, pk);
       }
-      l_run += rs;
+      l_run += (su[0] + su[1]) + (su[2] + su[3]);
+      l_o += (sr[0] + sr[1]) + (sr[2] + sr[3]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
@@ -307,7 +326,7 @@ __global__ void __launch_bounds__(384, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-        const float inv = 1.f / l_run;
+        const float inv = 1.f / l_o;
         const size_t grow = static_cast<size_t>(bh) * Nq + static_cast<size_t>(qt) * kTile + row;
         uint4* dst = reinterpret_cast<uint4*>(o_ptr + grow * D);
 #pragma unroll 1
