@@ -136,6 +136,42 @@ attn_status dispatch_bwd_causal(int causal, const CUtensorMap& mq, const CUtenso
 
 }  // namespace
 
+// ------------------------------------------------ allocation-free backward
+//
+// attn_bwd_noalloc runs the backward pass with its workspace in this fixed
+// array instead of a caller-provided buffer.  It exists for callers that
+// cannot allocate device memory when they call: a plugin inside another
+// runtime's execution callback that must not allocate, or a process whose
+// device memory is entirely held by another allocator's pool.  The array is
+// part of this library's module, so every GPU that loads the library holds
+// it until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(72) << 20;  // 72 MiB
+static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// In host code g_bwd_scratch is only a host-side stand-in for the device
+// array: its device address is looked up once per device, with that device
+// current, and cached.
+attn_status scratch_for_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr) return ATTN_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
@@ -203,6 +239,25 @@ attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const vo
               : dispatch_bwd_causal<128, false>(causal, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st);
 }
 
+attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                             const void* dout, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d,
+                             float scale, int causal, attn_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
+  if (cs != ATTN_OK) return cs;
+  if (attn_bwd_workspace_bytes(B, H, Nq, Nk, d) > kNoAllocScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  const attn_status ss = scratch_for_current_device(&scratch);
+  if (ss != ATTN_OK) return ss;
+  // The preprocess kernel rewrites every byte of the scratch that the main
+  // kernel reads (it zeroes the dQ accumulator), so the previous call's
+  // contents never leak into this one.
+  return attn_bwd_phase(q, k, v, o, lse, dout, dq, dk, dv, scratch, B, H, Nq, Nk, d, scale, causal, dtype,
+                        ATTN_BWD_ALL, stream);
+}
+
+size_t attn_bwd_noalloc_max_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
 attn_status attn_last_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
   int status = 0;
@@ -221,6 +276,7 @@ const char* attn_status_string(attn_status s) {
     case ATTN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
     case ATTN_ERR_CUDA: return "CUDA error";
     case ATTN_ERR_TIMEOUT: return "device wait timed out";
+    case ATTN_ERR_SCRATCH_LIMIT: return "problem needs more scratch than attn_bwd_noalloc's fixed 72 MiB array";
   }
   return "unknown status";
 }

@@ -19,7 +19,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libattn.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "attn.h")
 
-ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(5)
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_SCRATCH_LIMIT = range(6)
 ATTN_FP16, ATTN_BF16 = 0, 1
 ATTN_BWD_ALL, ATTN_BWD_PREPROCESS, ATTN_BWD_MAIN, ATTN_BWD_CONVERT = range(4)
 
@@ -49,6 +49,10 @@ def load() -> ctypes.CDLL:
     lib.attn_bwd.restype = st
     lib.attn_bwd_phase.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
     lib.attn_bwd_phase.restype = st
+    lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+    lib.attn_bwd_noalloc.restype = st
+    lib.attn_bwd_noalloc_max_scratch_bytes.argtypes = []
+    lib.attn_bwd_noalloc_max_scratch_bytes.restype = ctypes.c_size_t
     lib.attn_last_device_status.argtypes = [vp]
     lib.attn_last_device_status.restype = st
     lib.attn_status_string.argtypes = [st]
@@ -90,6 +94,18 @@ def attn_bwd_phase(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d
     """Direct call of attn_bwd_phase (one of the three backward kernels)."""
     return load().attn_bwd_phase(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale,
                                  int(causal), dtype, phase, stream)
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
+    """Direct call of attn_bwd_noalloc: the backward pass with the library's
+    fixed scratch array as workspace, for callers that cannot allocate device
+    memory when they call (see include/attn.h)."""
+    return load().attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, Nq, Nk, d, scale, int(causal), dtype,
+                                   stream)
+
+
+def attn_bwd_noalloc_max_scratch_bytes() -> int:
+    return int(load().attn_bwd_noalloc_max_scratch_bytes())
 
 
 def attn_bwd_workspace_bytes(B, H, Nq, Nk, d) -> int:

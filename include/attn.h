@@ -54,7 +54,8 @@ typedef enum {
   ATTN_ERR_INVALID_ARG = 1,
   ATTN_ERR_UNSUPPORTED = 2,
   ATTN_ERR_CUDA = 3,
-  ATTN_ERR_TIMEOUT = 4
+  ATTN_ERR_TIMEOUT = 4,
+  ATTN_ERR_SCRATCH_LIMIT = 5
 } attn_status;
 
 typedef enum { ATTN_FP16 = 0, ATTN_BF16 = 1 } attn_dtype;
@@ -126,6 +127,36 @@ attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const vo
                            const float* lse, const void* dout, void* dq, void* dk, void* dv,
                            void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
                            int causal, attn_dtype dtype, int phase, void* stream);
+
+/*
+ * attn_bwd without a workspace argument.  The paper has no counterpart: this
+ * entry point exists for callers that cannot allocate device memory when
+ * they call -- a plugin running inside another runtime's execution callback,
+ * where allocating is not allowed, or a process whose device memory is all
+ * held by another allocator's pool.  It allocates nothing: the workspace is
+ * a fixed 72 MiB array inside the library (every GPU that loads the library
+ * holds it until the process exits), and the caller still passes every input
+ * and output.
+ *   Limit.  Problems whose attn_bwd_workspace_bytes() exceeds
+ *           attn_bwd_noalloc_max_scratch_bytes() (72 MiB; e.g. B*H*Nq up
+ *           to 145,187 rows at d = 128) return ATTN_ERR_SCRATCH_LIMIT
+ *           before any work is enqueued.
+ *   Set-up. The first call on each device looks up the array's device
+ *           address (cudaGetSymbolAddress) with that device current; make
+ *           that first call before any stream capture.
+ *   Sharing. Every call on a device uses the same array, which keeps the
+ *           last call's contents; each call clears what must start at zero.
+ *           Calls whose kernels overlap on the GPU (e.g. on two streams)
+ *           race on the array and give wrong results: order them.
+ * Arguments, results and other errors as for attn_bwd.
+ */
+attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                             attn_dtype dtype, void* stream);
+
+/* Size in bytes of attn_bwd_noalloc's fixed scratch array (72 MiB). */
+size_t attn_bwd_noalloc_max_scratch_bytes(void);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word that
