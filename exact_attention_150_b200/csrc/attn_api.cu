@@ -102,7 +102,7 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     auto kern = attn::bwd_main_kernel<D, BF16, CAUSAL>;
     if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
     dim3 grid(BH, Nk / kTile);
-    kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, dqacc, static_cast<uint16_t*>(dk),
+    kern<<<grid, 512, L::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, dqacc, static_cast<uint16_t*>(dk),
                                        static_cast<uint16_t*>(dv), Nq, Nk, scale, scale * 1.4426950408889634f);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }

@@ -15,17 +15,28 @@
 //                       dK_j += dS^T Q_i              (A = dS^T from TMEM)
 //                       dQacc_i += scale * dS K_j     (fp32 atomics)
 //                     then dK_j = scale * dK_j and dV_j are written once.
+//                     (dQ is formed transposed, dQ^T = K_j^T dS^T, when
+//                     d = 128, so that the atomics of a warp cover one
+//                     contiguous 128-byte row segment.)
 //   bwd_post_kernel   dQ = 16-bit(dQacc)
 //
-// Main-kernel CTA layout (384 threads):
-//   warp 0      TMA producer (K_j, V_j once; Q_i, dO_i through 2 stages)
-//   warp 1      MMA issuer (one thread)
-//   warp 2      TMEM allocation
-//   warps 4-7   P / dS computation, thread = key row = TMEM lane
-//   warps 8-11  dQ drain (thread = query row), then the dK/dV epilogue
-// Tensor memory: [0,128) S^T (P^T packed in [0,64)), [128,256) dP^T (dS^T
-// packed in [128,192)), [256,256+D) dV, [256+D,256+2D) dK, and the dQ tile in
-// the columns freed by packing: [64,128) and [192,256) (64 columns each).
+// Main-kernel CTA layout (512 threads, one CTA per SM):
+//   warp 0       TMA producer (K_j, V_j once; Q_i, dO_i through 2 stages)
+//   warp 1       MMA issuer (one thread)
+//   warp 2       TMEM allocation
+//   warps 4-7    P / dS for query columns [0, 64)   (thread = key row = TMEM lane)
+//   warps 8-11   P / dS for query columns [64, 128)
+//   warps 12-15  dQ drain, then the dK/dV epilogue
+// Tensor memory (d = 128):
+//   [0,128)    S^T fp32; overwritten in place by P^T (16-bit pairs) in
+//              [0,32) and [64,96) and by dS^T in [32,64) and [96,128)
+//   [128,256)  dP^T fp32, then dQ^T = K^T dS^T fp32 (lane = head-dim index)
+//   [256,384)  dV,  [384,512) dK
+// For d = 64 the dQ tile is dS K (lane = query row) in [128,192), dV in
+// [256,320) and dK in [320,384).
+// Per query tile the MMA issue order is  dP^T, dV, dK, S^T(next), dQ,  so
+// that the P pass and the dS pass of the softmax warps overlap the dP^T and
+// dV products, and the next tile's P pass overlaps this tile's dQ product.
 #pragma once
 
 #include "sm100.cuh"
@@ -45,8 +56,8 @@ struct BwdLayout {
   static constexpr int kDSOff = kStageOff + kStages * 2 * kTileBytes;
   static constexpr int kDSBytes = kBwdTile * kBwdTile * 2;
   static constexpr int kBarOff = kDSOff + kDSBytes;
-  // kv_full, qd_full[S], qd_empty[S], s_full, dp_full, ds_full, dq_full, dq_free, acc_full, mma_done
-  static constexpr int kNumBars = 1 + 2 * kStages + 7;
+  // kv_full, qd_full[S], qd_empty[S], s_full, dp_full, p_full, ds_full, dq_full, dq_free, acc_full, mma_done
+  static constexpr int kNumBars = 1 + 2 * kStages + 8;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -102,13 +113,15 @@ __global__ void __launch_bounds__(256)
 }
 
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const float* __restrict__ dvec, const float* __restrict__ nlse2, float* __restrict__ dqacc,
                     uint16_t* __restrict__ dk_ptr, uint16_t* __restrict__ dv_ptr, int Nq, int Nk, float scale,
                     float scale_log2) {
   using L = BwdLayout<D>;
+  constexpr bool kDqT = (D == 128);  // dQ formed transposed (see above)
+  constexpr uint32_t kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 256 + D;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -118,11 +131,12 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* qd_empty = qd_full + L::kStages;
   uint64_t* s_full = qd_empty + L::kStages;
   uint64_t* dp_full = s_full + 1;
-  uint64_t* ds_full = s_full + 2;
-  uint64_t* dq_full = s_full + 3;
-  uint64_t* dq_free = s_full + 4;
-  uint64_t* acc_full = s_full + 5;
-  uint64_t* mma_done = s_full + 6;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* ds_full = s_full + 3;
+  uint64_t* dq_full = s_full + 4;
+  uint64_t* dq_free = s_full + 5;
+  uint64_t* acc_full = s_full + 6;
+  uint64_t* mma_done = s_full + 7;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -142,7 +156,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(ds_full, 128);
+    mbar_init(p_full, 256);
+    mbar_init(ds_full, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 128);
     mbar_init(acc_full, 1);
@@ -198,115 +213,157 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);   // K-major x K-major
-      constexpr uint32_t kIdAcc = idesc_f16(BF16, 128, D, false, true);    // TMEM A x MN-major B
-      constexpr uint32_t kIdQ = idesc_f16(BF16, 128, 64, true, true);      // MN-major A x MN-major B
+      constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // K-major x K-major
+      constexpr uint32_t kIdAcc = idesc_f16(BF16, 128, D, false, true);   // TMEM A x MN-major B
+      // dQ^T = K^T dS^T (M = d) or dQ = dS K (M = queries); both operands MN-major.
+      constexpr uint32_t kIdQ = kDqT ? idesc_f16(BF16, 128, 128, true, true) : idesc_f16(BF16, 128, 64, true, true);
       const uint32_t k_addr = smem_u32(smem + L::kKOff);
       const uint32_t v_addr = smem_u32(smem + L::kVOff);
       const uint32_t ds_addr = smem_u32(smem + L::kDSOff);
-      bool ok = mbar_wait(kv_full, 0, abort_flag);
+      auto stage_addr = [&](int it) {
+        return smem_u32(smem + L::kStageOff + (it % L::kStages) * 2 * L::kTileBytes);
+      };
+      // Packed 16-bit P^T / dS^T columns of K step ks (16 queries).
+      auto p_col = [](int ks) { return static_cast<uint32_t>(64 * (ks >> 2) + 8 * (ks & 3)); };
+      auto issue_st = [&](uint32_t q_addr) {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
+          mma_ss(tmem, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), kIdS,
+                 ks > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_flag) && mbar_wait(&qd_full[0], 0, abort_flag);
+      if (ok && n_it > 0) {
+        tc_fence_after();
+        issue_st(stage_addr(0));
+        mma_commit(s_full);
+      }
       for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it % L::kStages;
-        const uint32_t q_addr = smem_u32(smem + L::kStageOff + s * 2 * L::kTileBytes);
+        const uint32_t q_addr = stage_addr(it);
         const uint32_t do_addr = q_addr + L::kTileBytes;
-        if (!mbar_wait(&qd_full[s], (it / L::kStages) & 1, abort_flag)) break;
-        // The dQ tile of the previous query tile occupies columns that S^T and
-        // dP^T overwrite: wait until it has been drained.
+        // dP^T overwrites the previous tile's dQ columns: wait for the drain.
         if (it > 0 && !mbar_wait(dq_free, (it - 1) & 1, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-          mma_ss(tmem + 0, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), kIdS,
-                 ks > 0 ? 1u : 0u);
-        }
-        mma_commit(s_full);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-          mma_ss(tmem + 128, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024), kIdS,
+          mma_ss(tmem + kColDP, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024), kIdS,
                  ks > 0 ? 1u : 0u);
         }
         mma_commit(dp_full);
+        if (!mbar_wait(p_full, it & 1, abort_flag)) break;
+        tc_fence_after();
+        // dV += P^T dO: A from TMEM, B = dO MN-major (16 query rows per K step).
+#pragma unroll
+        for (int ks = 0; ks < kBwdTile / 16; ++ks)
+          mma_ts(tmem + kColDV, tmem + p_col(ks), sdesc_sw128(do_addr + ks * 2048, L::kChunkBytes, 1024), kIdAcc,
+                 (it > 0 || ks > 0) ? 1u : 0u);
         if (!mbar_wait(ds_full, it & 1, abort_flag)) break;
         tc_fence_after();
-        // dV += P^T dO and dK += dS^T Q: A from TMEM (8 columns per 16 queries),
-        // B MN-major with 16 query rows (2048 bytes) per K step.
+        // dK += dS^T Q: A from TMEM, B = Q MN-major.
 #pragma unroll
         for (int ks = 0; ks < kBwdTile / 16; ++ks)
-          mma_ts(tmem + 256, tmem + 0 + ks * 8, sdesc_sw128(do_addr + ks * 2048, L::kChunkBytes, 1024), kIdAcc,
-                 (it > 0 || ks > 0) ? 1u : 0u);
-#pragma unroll
-        for (int ks = 0; ks < kBwdTile / 16; ++ks)
-          mma_ts(tmem + 256 + D, tmem + 128 + ks * 8, sdesc_sw128(q_addr + ks * 2048, L::kChunkBytes, 1024),
+          mma_ts(tmem + kColDK, tmem + 32 + p_col(ks), sdesc_sw128(q_addr + ks * 2048, L::kChunkBytes, 1024),
                  kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&qd_empty[s]);
-        // dQ_i = dS K_j, in 64-column halves of the head dimension.
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h)
-#pragma unroll
-          for (int ks = 0; ks < kBwdTile / 16; ++ks)
-            mma_ss(tmem + 64 + 128 * h, sdesc_sw128(ds_addr + ks * 2048, L::kChunkBytes, 1024),
-                   sdesc_sw128(k_addr + h * L::kChunkBytes + ks * 2048, L::kChunkBytes, 1024), kIdQ,
-                   ks > 0 ? 1u : 0u);
-        mma_commit(dq_full);
+        mma_commit(&qd_empty[it % L::kStages]);
         if (it == n_it - 1) mma_commit(acc_full);
+        // The next tile's S^T only overwrites P^T / dS^T, which dV and dK
+        // (issued above) have consumed; issuing it before dQ lets the next P
+        // pass overlap this tile's dQ product.
+        if (it + 1 < n_it) {
+          if (!mbar_wait(&qd_full[(it + 1) % L::kStages], ((it + 1) / L::kStages) & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_st(stage_addr(it + 1));
+          mma_commit(s_full);
+        }
+#pragma unroll
+        for (int ks = 0; ks < kBwdTile / 16; ++ks) {
+          if constexpr (kDqT)  // A = K^T (M = d), B = dS^T (N = queries)
+            mma_ss(tmem + kColDQ, sdesc_sw128(k_addr + ks * 2048, L::kChunkBytes, 1024),
+                   sdesc_sw128(ds_addr + ks * 2048, L::kChunkBytes, 1024), kIdQ, ks > 0 ? 1u : 0u);
+          else  // A = dS (M = queries), B = K (N = d)
+            mma_ss(tmem + kColDQ, sdesc_sw128(ds_addr + ks * 2048, L::kChunkBytes, 1024),
+                   sdesc_sw128(k_addr + ks * 2048, L::kChunkBytes, 1024), kIdQ, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(dq_full);
       }
       mma_commit(mma_done);
       mbar_drain(mma_done, 0);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ P and dS
+    const int h = (warp - 4) >> 2;  // query columns [64h, 64h + 64)
     const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // key row within tile j = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    uint8_t* ds_row = smem + L::kDSOff + r * 128;
+    const int r = wq * 32 + lane;   // key row within tile j = TMEM lane
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    uint8_t* ds_row = smem + L::kDSOff + h * L::kChunkBytes + r * 128;
     for (int it = 0; it < n_it; ++it) {
       const int i = i0 + it;
-      bool ok = mbar_wait(s_full, it & 1, abort_flag);
-      ok = ok && mbar_wait(dp_full, it & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      const bool diag = CAUSAL && i == j;
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag))) break;
       tc_fence_after();
-      const size_t vbase = static_cast<size_t>(bh) * Nq + static_cast<size_t>(i) * kBwdTile;
+      const size_t vbase = static_cast<size_t>(bh) * Nq + static_cast<size_t>(i) * kBwdTile + 64 * h;
       const float4* nl4 = reinterpret_cast<const float4*>(nlse2 + vbase);
       const float4* dd4 = reinterpret_cast<const float4*>(dvec + vbase);
-#pragma unroll 1
-      for (int c = 0; c < kBwdTile / 16; ++c) {
-        uint32_t sr[16], pr[16];
-        tmem_ld16(tmem + lane_off + c * 16, sr);
-        tmem_ld16(tmem + lane_off + 128 + c * 16, pr);
-        float nl[16], dd[16];
+      // P pass: P^T = exp2(S^T * scale * log2e - LSE * log2e), packed 16-bit.
+      uint32_t ppk[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[16];
+        tmem_ld16(t_row + 64 * h + 16 * c, sr);
+        float nl[16];
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          const float4 a = nl4[c * 4 + v];
-          const float4 b = dd4[c * 4 + v];
+          const float4 a = nl4[4 * c + v];
           nl[4 * v] = a.x; nl[4 * v + 1] = a.y; nl[4 * v + 2] = a.z; nl[4 * v + 3] = a.w;
-          dd[4 * v] = b.x; dd[4 * v + 1] = b.y; dd[4 * v + 2] = b.z; dd[4 * v + 3] = b.w;
         }
-        uint32_t ppk[8], dpk[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
           float p0 = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, nl[e]));
           float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), scale_log2, nl[e + 1]));
-          if (CAUSAL && i == j) {
-            // key r is visible to query q iff r <= q
-            if (r > c * 16 + e) p0 = 0.f;
-            if (r > c * 16 + e + 1) p1 = 0.f;
+          if (diag) {  // key r is visible to query q iff r <= q
+            const int q = 64 * h + 16 * c + e;
+            if (r > q) p0 = 0.f;
+            if (r > q + 1) p1 = 0.f;
           }
-          const float d0 = p0 * (__uint_as_float(pr[e]) - dd[e]);
-          const float d1 = p1 * (__uint_as_float(pr[e + 1]) - dd[e + 1]);
-          ppk[e / 2] = pack2<BF16>(p0, p1);
-          dpk[e / 2] = pack2<BF16>(d0, d1);
+          ppk[8 * c + e / 2] = pack2<BF16>(p0, p1);
         }
-        tmem_st8(tmem + lane_off + c * 8, ppk);
-        tmem_st8(tmem + lane_off + 128 + c * 8, dpk);
-        // dS^T row r, queries [16c, 16c+16): two 16-byte units of the
-        // 128-byte-swizzled MN-major tile (64 queries per 16 KB chunk).
-        uint8_t* chunk_row = ds_row + (c >> 2) * L::kChunkBytes;
+        if (c & 1) {
+          uint32_t out[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) out[e] = ppk[8 * (c - 1) + e];
+          tmem_st16(t_row + 64 * h + 16 * (c >> 1), out);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      // dS pass: dS^T = P^T * (dP^T - D), packed into TMEM and into the
+      // 128-byte-swizzled shared tile (row r, 64 queries per 16 KB chunk).
+      if (!__all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pr[16];
+        tmem_ld16(t_row + kColDP + 64 * h + 16 * c, pr);
+        float dd[16];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float4 b = dd4[4 * c + v];
+          dd[4 * v] = b.x; dd[4 * v + 1] = b.y; dd[4 * v + 2] = b.z; dd[4 * v + 3] = b.w;
+        }
+        uint32_t dpk[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const float2 p = unpack2<BF16>(ppk[8 * c + e / 2]);
+          dpk[e / 2] = pack2<BF16>(p.x * (__uint_as_float(pr[e]) - dd[e]), p.y * (__uint_as_float(pr[e + 1]) - dd[e + 1]));
+        }
+        tmem_st8(t_row + 64 * h + 32 + 8 * c, dpk);
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
-          const int unit = ((c & 3) * 2 + v) ^ (r & 7);
-          *reinterpret_cast<uint4*>(chunk_row + unit * 16) =
+          const int unit = (2 * c + v) ^ (r & 7);
+          *reinterpret_cast<uint4*>(ds_row + unit * 16) =
               make_uint4(dpk[4 * v], dpk[4 * v + 1], dpk[4 * v + 2], dpk[4 * v + 3]);
         }
       }
@@ -315,50 +372,75 @@ __global__ void __launch_bounds__(384, 1)
       fence_proxy_async_smem();
       mbar_arrive(ds_full);
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 12) {
     // ------------------------------------------------------------ dQ drain, dK/dV epilogue
     const int wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const int row = wq * 32 + lane;  // TMEM lane: head-dim index (dQ^T) or query row (dQ)
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      ok = mbar_wait(dq_full, it & 1, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
+      ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float* dst = dqacc + (static_cast<size_t>(bh) * Nq + static_cast<size_t>(i0 + it) * kBwdTile + row) * D;
-#pragma unroll 1
-      for (int h = 0; h < D / 64; ++h) {
+      const size_t qrow0 = static_cast<size_t>(bh) * Nq + static_cast<size_t>(i0 + it) * kBwdTile;
+      if constexpr (kDqT) {
+        // Thread = head-dim index d; a warp's reduction covers 32 consecutive
+        // d of one query row (128 contiguous bytes).
+        float* base = dqacc + qrow0 * D + row;
+        uint32_t va[32], vb[32];
+        tmem_ld32(t_row + kColDQ, va);
+        tmem_ld32(t_row + kColDQ + 32, vb);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(tmem + lane_off + 64 + 128 * h + 32 * c, rr);
+        for (int q = 0; q < 32; ++q) atomicAdd(base + static_cast<size_t>(q) * D, __uint_as_float(va[q]) * scale);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            atomicAdd(reinterpret_cast<float4*>(dst + h * 64 + c * 32 + 4 * v),
-                      make_float4(__uint_as_float(rr[4 * v]) * scale, __uint_as_float(rr[4 * v + 1]) * scale,
-                                  __uint_as_float(rr[4 * v + 2]) * scale, __uint_as_float(rr[4 * v + 3]) * scale));
-        }
+        for (int q = 0; q < 32; ++q)
+          atomicAdd(base + static_cast<size_t>(32 + q) * D, __uint_as_float(vb[q]) * scale);
+        tmem_ld32(t_row + kColDQ + 64, va);
+        tmem_ld32(t_row + kColDQ + 96, vb);
+        tc_fence_before();
+        mbar_arrive(dq_free);
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          atomicAdd(base + static_cast<size_t>(64 + q) * D, __uint_as_float(va[q]) * scale);
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          atomicAdd(base + static_cast<size_t>(96 + q) * D, __uint_as_float(vb[q]) * scale);
+      } else {
+        // Thread = query row; 64 head-dim values as 16-byte vector reductions.
+        uint32_t va[32], vb[32];
+        tmem_ld32(t_row + kColDQ, va);
+        tmem_ld32(t_row + kColDQ + 32, vb);
+        tc_fence_before();
+        mbar_arrive(dq_free);
+        float* dst = dqacc + (qrow0 + row) * D;
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          atomicAdd(reinterpret_cast<float4*>(dst + 4 * v),
+                    make_float4(__uint_as_float(va[4 * v]) * scale, __uint_as_float(va[4 * v + 1]) * scale,
+                                __uint_as_float(va[4 * v + 2]) * scale, __uint_as_float(va[4 * v + 3]) * scale));
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          atomicAdd(reinterpret_cast<float4*>(dst + 32 + 4 * v),
+                    make_float4(__uint_as_float(vb[4 * v]) * scale, __uint_as_float(vb[4 * v + 1]) * scale,
+                                __uint_as_float(vb[4 * v + 2]) * scale, __uint_as_float(vb[4 * v + 3]) * scale));
       }
-      tc_fence_before();
-      mbar_arrive(dq_free);
     }
     if (ok && n_it > 0) {
-      ok = mbar_wait(acc_full, 0, abort_flag);
-      if (__all_sync(0xffffffffu, ok)) {
+      if (__all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag))) {
         tc_fence_after();
+        // dK / dV: M = keys, so the TMEM lane is the key row.
         const size_t grow = static_cast<size_t>(bh) * Nk + static_cast<size_t>(j) * kBwdTile + row;
         uint4* dvd = reinterpret_cast<uint4*>(dv_ptr + grow * D);
         uint4* dkd = reinterpret_cast<uint4*>(dk_ptr + grow * D);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t rv[32], pk[16];
-          tmem_ld32(tmem + lane_off + 256 + c * 32, rv);
+          tmem_ld32(t_row + kColDV + c * 32, rv);
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack2<BF16>(__uint_as_float(rv[2 * e]), __uint_as_float(rv[2 * e + 1]));
 #pragma unroll
           for (int v = 0; v < 4; ++v) dvd[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-          tmem_ld32(tmem + lane_off + 256 + D + c * 32, rv);
+          tmem_ld32(t_row + kColDK + c * 32, rv);
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             pk[e] = pack2<BF16>(__uint_as_float(rv[2 * e]) * scale, __uint_as_float(rv[2 * e + 1]) * scale);
