@@ -276,6 +276,7 @@ const char* attn_status_string(attn_status s) {
     case ATTN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
     case ATTN_ERR_CUDA: return "CUDA error";
     case ATTN_ERR_TIMEOUT: return "device wait timed out";
+    case ATTN_ERR_SMEM: return "kernel found less shared memory than its tiles need";
     case ATTN_ERR_SCRATCH_LIMIT: return "problem needs more scratch than attn_bwd_noalloc's fixed 72 MiB array";
   }
   return "unknown status";

@@ -55,13 +55,19 @@ struct BwdLayout {
   static constexpr int kStageOff = 2 * kTileBytes;  // stage s: Q at +s*2T, dO at +s*2T+T
   static constexpr int kDSOff = kStageOff + kStages * 2 * kTileBytes;
   static constexpr int kDSBytes = kBwdTile * kBwdTile * 2;
-  static constexpr int kBarOff = kDSOff + kDSBytes;
+  // Per stage: -log2(e) LSE and D of the stage's 128 query rows (512 B each).
+  static constexpr int kVecOff = kDSOff + kDSBytes;
+  static constexpr int kVecBytes = 2 * kBwdTile * 4;
+  static constexpr int kBarOff = kVecOff + kStages * kVecBytes;
   // kv_full, qd_full[S], qd_empty[S], s_full, dp_full, p_full, ds_full, dq_full, dq_free, acc_full, mma_done
   static constexpr int kNumBars = 1 + 2 * kStages + 8;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
-  static constexpr int kAlloc = kBytes + 1024;
-  static_assert(kAlloc <= 232448, "shared memory budget");
+  // The tiles need a 1024-byte aligned base.  The dynamic shared window
+  // starts 1024-byte aligned in practice; the slack below covers what the
+  // 227 KB limit leaves, and the kernel checks the real need at entry.
+  static constexpr int kAlloc = kBytes + 1024 <= 232448 ? kBytes + 1024 : 232448;
+  static_assert(kBytes <= 232448, "shared memory budget");
 };
 
 // One group of D/8 threads per row; each thread handles 8 elements.
@@ -148,6 +154,12 @@ __global__ void __launch_bounds__(512, 1)
   const int i0 = CAUSAL ? j : 0;
   const int n_it = nqt - i0;
 
+  // Refuse to run (and report) if alignment left too little shared memory.
+  if (static_cast<uint32_t>(smem - smem_raw) + L::kBytes > dynamic_smem_bytes()) {
+    if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusSmem);
+    return;
+  }
+
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < L::kStages; ++s) {
@@ -197,12 +209,15 @@ __global__ void __launch_bounds__(512, 1)
           break;
         }
         const int qrow = bh * Nq + (i0 + it) * kBwdTile;
-        mbar_arrive_expect_tx(&qd_full[s], 2 * L::kTileBytes);
+        mbar_arrive_expect_tx(&qd_full[s], 2 * L::kTileBytes + L::kVecBytes);
         uint8_t* qdst = smem + L::kStageOff + s * 2 * L::kTileBytes;
         for (int c = 0; c < D / 64; ++c) {
           tma_load_2d(qdst + c * L::kChunkBytes, &tm_q, &qd_full[s], c * 64, qrow);
           tma_load_2d(qdst + L::kTileBytes + c * L::kChunkBytes, &tm_do, &qd_full[s], c * 64, qrow);
         }
+        uint8_t* vdst = smem + L::kVecOff + s * L::kVecBytes;
+        bulk_load(vdst, nlse2 + qrow, kBwdTile * 4, &qd_full[s]);
+        bulk_load(vdst + kBwdTile * 4, dvec + qrow, kBwdTile * 4, &qd_full[s]);
       }
       if (!ok) {
         mbar_drain(kv_full, 0);
@@ -303,9 +318,11 @@ __global__ void __launch_bounds__(512, 1)
       const bool diag = CAUSAL && i == j;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag))) break;
       tc_fence_after();
-      const size_t vbase = static_cast<size_t>(bh) * Nq + static_cast<size_t>(i) * kBwdTile + 64 * h;
-      const float4* nl4 = reinterpret_cast<const float4*>(nlse2 + vbase);
-      const float4* dd4 = reinterpret_cast<const float4*>(dvec + vbase);
+      // -log2(e) LSE and D of this warpgroup's 64 queries, staged by the
+      // producer with the stage's Q and dO (read as shared-memory broadcasts).
+      const float4* nl4 =
+          reinterpret_cast<const float4*>(smem + L::kVecOff + (it % L::kStages) * L::kVecBytes) + 16 * h;
+      const float4* dd4 = nl4 + kBwdTile / 4;
       // P pass: P^T = exp2(S^T * scale * log2e - LSE * log2e), packed 16-bit.
       uint32_t ppk[32];
 #pragma unroll

@@ -16,6 +16,7 @@ namespace attn {
 
 // Status codes mirrored from attn.h (kept numeric to avoid a header cycle).
 constexpr int kStatusTimeout = 4;
+constexpr int kStatusSmem = 6;
 
 // Device status word: 0 = OK, otherwise an attn_status code.
 __device__ int g_device_status;
@@ -112,6 +113,23 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// Contiguous (untiled) bulk copy global -> shared; both addresses 16-byte
+// aligned, `bytes` a multiple of 16.  Completion counts as transaction bytes
+// on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Dynamic shared memory actually granted to this CTA, in bytes.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t v;
+  asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));
+  return v;
 }
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (tcgen05).

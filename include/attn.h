@@ -38,7 +38,9 @@
  *   written to any output when a call returns an error.  There is no fallback
  *   to another implementation.  Kernels never trap: a wait inside a kernel
  *   that exceeds its time limit makes the kernel record ATTN_ERR_TIMEOUT in a
- *   device status word and return early; attn_last_device_status() reads it.
+ *   device status word and return early, and a kernel that finds less shared
+ *   memory than its tiles need records ATTN_ERR_SMEM and returns without
+ *   work; attn_last_device_status() reads the word.
  */
 #ifndef ATTN_H_
 #define ATTN_H_
@@ -55,7 +57,8 @@ typedef enum {
   ATTN_ERR_UNSUPPORTED = 2,
   ATTN_ERR_CUDA = 3,
   ATTN_ERR_TIMEOUT = 4,
-  ATTN_ERR_SCRATCH_LIMIT = 5
+  ATTN_ERR_SCRATCH_LIMIT = 5,
+  ATTN_ERR_SMEM = 6
 } attn_status;
 
 typedef enum { ATTN_FP16 = 0, ATTN_BF16 = 1 } attn_dtype;
