@@ -12,7 +12,7 @@
 //                       P^T  = exp2(S^T * scale*log2e - LSE_i*log2e)
 //                       dS^T = P^T * (dP^T - D_i)
 //                       dV_j += P^T dO_i              (A = P^T from TMEM)
-//                       dK_j += dS^T Q_i              (A = dS^T from TMEM)
+//                       dK_j += dS^T Q_i              (A = dS^T from shared memory)
 //                       dQacc_i += scale * dS K_j     (fp32 atomics)
 //                     then dK_j = scale * dK_j and dV_j are written once.
 //                     (dQ is formed transposed, dQ^T = K_j^T dS^T, when
@@ -29,14 +29,18 @@
 //   warps 12-15  dQ drain, then the dK/dV epilogue
 // Tensor memory (d = 128):
 //   [0,128)    S^T fp32; overwritten in place by P^T (16-bit pairs) in
-//              [0,32) and [64,96) and by dS^T in [32,64) and [96,128)
+//              [0,32) and [64,96)
 //   [128,256)  dP^T fp32, then dQ^T = K^T dS^T fp32 (lane = head-dim index)
 //   [256,384)  dV,  [384,512) dK
 // For d = 64 the dQ tile is dS K (lane = query row) in [128,192), dV in
 // [256,320) and dK in [320,384).
-// Per query tile the MMA issue order is  dP^T, dV, dK, S^T(next), dQ,  so
-// that the P pass and the dS pass of the softmax warps overlap the dP^T and
-// dV products, and the next tile's P pass overlaps this tile's dQ product.
+// dS^T lives only in shared memory (128-byte swizzled, [key][query]): it is
+// the K-major A operand of dK += dS^T Q and an MN-major operand of the dQ
+// product.  Keeping it out of TMEM lets the next query tile's S^T be issued
+// right after dV, so per query tile the MMA issue order is
+//   dP^T, dV, S^T(next), dK, dQ
+// and the softmax warps go from this tile's dS pass straight to the next
+// tile's P pass while dK and dQ run on the tensor core.
 #pragma once
 
 #include "sm100.cuh"
@@ -230,6 +234,7 @@ __global__ void __launch_bounds__(512, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // K-major x K-major
       constexpr uint32_t kIdAcc = idesc_f16(BF16, 128, D, false, true);   // TMEM A x MN-major B
+      constexpr uint32_t kIdDK = idesc_f16(BF16, 128, D, false, true);    // K-major smem A x MN-major B
       // dQ^T = K^T dS^T (M = d) or dQ = dS K (M = queries); both operands MN-major.
       constexpr uint32_t kIdQ = kDqT ? idesc_f16(BF16, 128, 128, true, true) : idesc_f16(BF16, 128, 64, true, true);
       const uint32_t k_addr = smem_u32(smem + L::kKOff);
@@ -274,24 +279,25 @@ __global__ void __launch_bounds__(512, 1)
         for (int ks = 0; ks < kBwdTile / 16; ++ks)
           mma_ts(tmem + kColDV, tmem + p_col(ks), sdesc_sw128(do_addr + ks * 2048, L::kChunkBytes, 1024), kIdAcc,
                  (it > 0 || ks > 0) ? 1u : 0u);
-        if (!mbar_wait(ds_full, it & 1, abort_flag)) break;
-        tc_fence_after();
-        // dK += dS^T Q: A from TMEM, B = Q MN-major.
-#pragma unroll
-        for (int ks = 0; ks < kBwdTile / 16; ++ks)
-          mma_ts(tmem + kColDK, tmem + 32 + p_col(ks), sdesc_sw128(q_addr + ks * 2048, L::kChunkBytes, 1024),
-                 kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&qd_empty[it % L::kStages]);
-        if (it == n_it - 1) mma_commit(acc_full);
-        // The next tile's S^T only overwrites P^T / dS^T, which dV and dK
-        // (issued above) have consumed; issuing it before dQ lets the next P
-        // pass overlap this tile's dQ product.
+        // The next tile's S^T only overwrites P^T, which dV (issued above)
+        // consumes first; issuing it now lets the softmax warps move on to
+        // the next P pass as soon as this tile's dS pass is done.
         if (it + 1 < n_it) {
           if (!mbar_wait(&qd_full[(it + 1) % L::kStages], ((it + 1) / L::kStages) & 1, abort_flag)) break;
           tc_fence_after();
           issue_st(stage_addr(it + 1));
           mma_commit(s_full);
         }
+        if (!mbar_wait(ds_full, it & 1, abort_flag)) break;
+        tc_fence_after();
+        // dK += dS^T Q: A = dS^T K-major in shared memory (16 queries = 32
+        // bytes per K step, 4 steps per 64-query chunk), B = Q MN-major.
+#pragma unroll
+        for (int ks = 0; ks < kBwdTile / 16; ++ks)
+          mma_ss(tmem + kColDK, sdesc_sw128(ds_addr + (ks >> 2) * L::kChunkBytes + (ks & 3) * 32, 16, 1024),
+                 sdesc_sw128(q_addr + ks * 2048, L::kChunkBytes, 1024), kIdDK, (it > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&qd_empty[it % L::kStages]);
+        if (it == n_it - 1) mma_commit(acc_full);
 #pragma unroll
         for (int ks = 0; ks < kBwdTile / 16; ++ks) {
           if constexpr (kDqT)  // A = K^T (M = d), B = dS^T (N = queries)
@@ -319,72 +325,77 @@ __global__ void __launch_bounds__(512, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag))) break;
       tc_fence_after();
       // -log2(e) LSE and D of this warpgroup's 64 queries, staged by the
-      // producer with the stage's Q and dO (read as shared-memory broadcasts).
-      const float4* nl4 =
-          reinterpret_cast<const float4*>(smem + L::kVecOff + (it % L::kStages) * L::kVecBytes) + 16 * h;
-      const float4* dd4 = nl4 + kBwdTile / 4;
+      // producer with the stage's Q and dO.  Each lane reads two of each
+      // (coalesced); the inner loops broadcast them with warp shuffles, so
+      // no shared-memory access sits on their critical path.
+      const float* vec = reinterpret_cast<const float*>(smem + L::kVecOff + (it % L::kStages) * L::kVecBytes);
+      const float nl_lo = vec[64 * h + lane], nl_hi = vec[64 * h + 32 + lane];
+      const float dd_lo = vec[kBwdTile + 64 * h + lane], dd_hi = vec[kBwdTile + 64 * h + 32 + lane];
       // P pass: P^T = exp2(S^T * scale * log2e - LSE * log2e), packed 16-bit.
       uint32_t ppk[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[16];
-        tmem_ld16(t_row + 64 * h + 16 * c, sr);
-        float nl[16];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(t_row + 64 * h + 32 * c, sr);
+        const float nl_src = c ? nl_hi : nl_lo;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const float4 a = nl4[4 * c + v];
-          nl[4 * v] = a.x; nl[4 * v + 1] = a.y; nl[4 * v + 2] = a.z; nl[4 * v + 3] = a.w;
-        }
+        for (int g = 0; g < 2; ++g) {
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, nl[e]));
-          float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), scale_log2, nl[e + 1]));
-          if (diag) {  // key r is visible to query q iff r <= q
-            const int q = 64 * h + 16 * c + e;
-            if (r > q) p0 = 0.f;
-            if (r > q + 1) p1 = 0.f;
+          for (int e = 0; e < 16; e += 2) {
+            const int x = 16 * g + e;
+            const float n0 = __shfl_sync(0xffffffffu, nl_src, x);
+            const float n1 = __shfl_sync(0xffffffffu, nl_src, x + 1);
+            float p0 = ex2(fmaf(__uint_as_float(sr[x]), scale_log2, n0));
+            float p1 = ex2(fmaf(__uint_as_float(sr[x + 1]), scale_log2, n1));
+            if (diag) {  // key r is visible to query q iff r <= q
+              const int q = 64 * h + 32 * c + x;
+              if (r > q) p0 = 0.f;
+              if (r > q + 1) p1 = 0.f;
+            }
+            ppk[16 * c + x / 2] = pack2<BF16>(p0, p1);
           }
-          ppk[8 * c + e / 2] = pack2<BF16>(p0, p1);
         }
-        if (c & 1) {
+        if (c == 1) {
           uint32_t out[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) out[e] = ppk[8 * (c - 1) + e];
-          tmem_st16(t_row + 64 * h + 16 * (c >> 1), out);
+          for (int e = 0; e < 16; ++e) out[e] = ppk[e];
+          tmem_st16(t_row + 64 * h, out);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) out[e] = ppk[16 + e];
+          tmem_st16(t_row + 64 * h + 16, out);
         }
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
-      // dS pass: dS^T = P^T * (dP^T - D), packed into TMEM and into the
-      // 128-byte-swizzled shared tile (row r, 64 queries per 16 KB chunk).
+      // dS pass: dS^T = P^T * (dP^T - D), packed 16-bit into the 128-byte-
+      // swizzled shared tile (row r, 64 queries per 16 KB chunk).
       if (!__all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag))) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pr[16];
-        tmem_ld16(t_row + kColDP + 64 * h + 16 * c, pr);
-        float dd[16];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pr[32];
+        tmem_ld32(t_row + kColDP + 64 * h + 32 * c, pr);
+        const float dd_src = c ? dd_hi : dd_lo;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const float4 b = dd4[4 * c + v];
-          dd[4 * v] = b.x; dd[4 * v + 1] = b.y; dd[4 * v + 2] = b.z; dd[4 * v + 3] = b.w;
-        }
-        uint32_t dpk[8];
+        for (int g = 0; g < 2; ++g) {
+          uint32_t dpk[8];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const float2 p = unpack2<BF16>(ppk[8 * c + e / 2]);
-          dpk[e / 2] = pack2<BF16>(p.x * (__uint_as_float(pr[e]) - dd[e]), p.y * (__uint_as_float(pr[e + 1]) - dd[e + 1]));
-        }
-        tmem_st8(t_row + 64 * h + 32 + 8 * c, dpk);
+          for (int e = 0; e < 16; e += 2) {
+            const int x = 16 * g + e;
+            const float d0 = __shfl_sync(0xffffffffu, dd_src, x);
+            const float d1 = __shfl_sync(0xffffffffu, dd_src, x + 1);
+            const float2 p = unpack2<BF16>(ppk[16 * c + x / 2]);
+            dpk[e / 2] = pack2<BF16>(p.x * (__uint_as_float(pr[x]) - d0), p.y * (__uint_as_float(pr[x + 1]) - d1));
+          }
 #pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          const int unit = (2 * c + v) ^ (r & 7);
-          *reinterpret_cast<uint4*>(ds_row + unit * 16) =
-              make_uint4(dpk[4 * v], dpk[4 * v + 1], dpk[4 * v + 2], dpk[4 * v + 3]);
+          for (int v = 0; v < 2; ++v) {
+            const int unit = (4 * c + 2 * g + v) ^ (r & 7);
+            *reinterpret_cast<uint4*>(ds_row + unit * 16) =
+                make_uint4(dpk[4 * v], dpk[4 * v + 1], dpk[4 * v + 2], dpk[4 * v + 3]);
+          }
         }
       }
-      tmem_st_wait();
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(ds_full);
@@ -403,25 +414,27 @@ __global__ void __launch_bounds__(512, 1)
       if constexpr (kDqT) {
         // Thread = head-dim index d; a warp's reduction covers 32 consecutive
         // d of one query row (128 contiguous bytes).
+        // All 128 columns are read before the columns are released, so the
+        // next dP^T product does not wait for the reductions.
         float* base = dqacc + qrow0 * D + row;
-        uint32_t va[32], vb[32];
+        uint32_t va[32], vb[32], vc[32], vd[32];
         tmem_ld32(t_row + kColDQ, va);
         tmem_ld32(t_row + kColDQ + 32, vb);
+        tmem_ld32(t_row + kColDQ + 64, vc);
+        tmem_ld32(t_row + kColDQ + 96, vd);
+        tc_fence_before();
+        mbar_arrive(dq_free);
 #pragma unroll
         for (int q = 0; q < 32; ++q) atomicAdd(base + static_cast<size_t>(q) * D, __uint_as_float(va[q]) * scale);
 #pragma unroll
         for (int q = 0; q < 32; ++q)
           atomicAdd(base + static_cast<size_t>(32 + q) * D, __uint_as_float(vb[q]) * scale);
-        tmem_ld32(t_row + kColDQ + 64, va);
-        tmem_ld32(t_row + kColDQ + 96, vb);
-        tc_fence_before();
-        mbar_arrive(dq_free);
 #pragma unroll
         for (int q = 0; q < 32; ++q)
-          atomicAdd(base + static_cast<size_t>(64 + q) * D, __uint_as_float(va[q]) * scale);
+          atomicAdd(base + static_cast<size_t>(64 + q) * D, __uint_as_float(vc[q]) * scale);
 #pragma unroll
         for (int q = 0; q < 32; ++q)
-          atomicAdd(base + static_cast<size_t>(96 + q) * D, __uint_as_float(vb[q]) * scale);
+          atomicAdd(base + static_cast<size_t>(96 + q) * D, __uint_as_float(vd[q]) * scale);
       } else {
         // Thread = query row; 64 head-dim values as 16-byte vector reductions.
         uint32_t va[32], vb[32];
