@@ -60,7 +60,7 @@ attn_status check_common(int B, int H, int Nq, int Nk, int d, int causal, attn_d
   const long long bh = static_cast<long long>(B) * H;
   // TMA row coordinates and grid dimensions are 32-bit.
   if (bh > 0x7fffffffLL || bh * Nq > 0x7fffffffLL || bh * Nk > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  if (Nq / (2 * kTile) + 1 > 65535 || Nk / kTile > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (Nq / kTile > 65535 || Nk / kTile > 65535) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 
@@ -75,9 +75,8 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   using L = attn::FwdLayout<D>;
   auto kern = attn::fwd_kernel<D, BF16, CAUSAL>;
   if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
-  const int pairs = (Nq / kTile + 1) / 2;
-  dim3 grid(BH, pairs);
-  kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, Nq, Nk, scale_log2, pairs);
+  dim3 grid(BH, Nq / kTile);
+  kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, Nq, Nk, scale_log2);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

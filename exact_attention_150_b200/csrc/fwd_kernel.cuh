@@ -1,6 +1,6 @@
 // fwd_kernel.cuh -- fused attention forward for sm_100a.
 //
-// Computes, for one (batch, head) slice and a pair of 128-row query tiles,
+// Computes, for one (batch, head) slice and one 128-row query tile,
 //   S = Q K^T (tcgen05 MMA into tensor memory), the online softmax over the
 //   key tiles (running row maximum m and row sum l, rescaling with exp2),
 //   P cast to 16-bit in tensor memory, O += P V (tcgen05 MMA with P read from
@@ -9,19 +9,33 @@
 // (part 2, tiling and kernel fusion) with the online softmax named on the
 // page "Flash Attention 落地评估" (section 4); S never leaves the SM.
 //
+// Both products read their A operand from tensor memory (Q for S = Q K^T,
+// P for O += P V) and stream only K or V from shared memory: an MMA whose
+// two operands both come from shared memory runs at about half rate on
+// B200, one with A in tensor memory at full rate.
+//
 // CTA layout (384 threads, one CTA per SM):
-//   warp 0       TMA producer: both Q tiles once, then K_j, V_j through a
-//                ring of shared-memory slots
-//   warp 1       MMA issuer (one thread): S_t = Q_t K_j^T, O_t += P_t V_j
+//   warp 0       TMA producer: Q once, then K_0, K_1, V_0, K_2, V_1, ...
+//                through a ring of shared-memory slots
+//   warp 1       MMA issuer (one thread)
 //   warp 2       tensor-memory allocation / release
-//   warps 4-7    softmax for query tile 0   (thread = query row = TMEM lane)
-//   warps 8-11   softmax for query tile 1
-// The two query tiles ping-pong: while one warpgroup exponentiates its
-// scores, the tensor core works on the other tile.
+//   warps 4-7    softmax for key columns [0, 64) of every key tile
+//   warps 8-11   softmax for key columns [64, 128)
+//                (thread = query row = TMEM lane; the two warpgroups
+//                exchange their partial row maxima through shared memory)
 //
 // Tensor memory (512 columns x 128 lanes x 32 bit):
-//   [0,128) S_0 (P_0 packed 16-bit in [0,64)), [128,256) S_1 (P_1),
-//   [256,256+D) O_0, [256+D,256+2D) O_1.
+//   [0, D/2)     Q, 16-bit pairs (A operand of S = Q K^T)
+//   [64, 192)    S buffer 0     [192, 320)  S buffer 1
+//                (P of a buffer is packed 16-bit in place: the warpgroup
+//                owning key columns [64h, 64h+64) writes their P into
+//                buffer columns [64h, 64h+32))
+//   [320, 320+D) O
+//   [320+D, 336+D) L = P 1: the row sums of the rounded 16-bit P that the
+//                O product uses, accumulated (and rescaled) like O, so that
+//                O / L is a weighted mean of V rows with weights summing to one
+// Issue order: S(0), S(1), then per key tile j: PV(j) and L(j), S(j+2) --
+// the softmax of tile j+1 overlaps these products.
 #pragma once
 
 #include "sm100.cuh"
@@ -32,75 +46,105 @@ constexpr int kTile = 128;  // rows of a query tile and of a key/value tile
 
 template <int D>
 struct FwdLayout {
-  static constexpr int kChunks = D / 64;            // 128-byte column chunks per row
+  static constexpr int kChunks = D / 64;            // 128-byte column chunks per row (>= 1)
   static constexpr int kChunkBytes = kTile * 128;   // one 128-row chunk
   static constexpr int kTileBytes = kTile * D * 2;  // one 128 x D 16-bit tile
-  static constexpr int kSlots = D == 128 ? 5 : 8;   // K/V ring slots
+  static constexpr int kSlots = D == 128 ? 5 : 10;  // K/V ring slots
   static constexpr int kQOff = 0;
-  static constexpr int kRingOff = kQOff + 2 * kTileBytes;
-  static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-  // q_full, kv_full[kSlots], kv_empty[kSlots], s_full[2], p_full[2], o_full[2], mma_done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 7;
+  static constexpr int kRingOff = kQOff + kTileBytes;
+  // Exchange between the two softmax warpgroups: row maxima
+  // [2 parity][2 warpgroups][128 rows], then row sums [2][2][128].
+  static constexpr int kXOff = kRingOff + kSlots * kTileBytes;
+  static constexpr int kXBytes = 2 * 2 * 2 * kTile * 4;
+  // 128 x 16 tile of ones (unswizzled K-major core matrices): B operand of
+  // the row-sum product L += P 1.
+  static constexpr int kOnesOff = kXOff + kXBytes;
+  static constexpr int kOnesBytes = kTile * 16 * 2;
+  static constexpr int kBarOff = kOnesOff + kOnesBytes;
+  // q_full, q_tmem, kv_full[kSlots], kv_empty[kSlots], s_full[2], p_full[2], pv_done, o_full, mma_done,
+  // xmax[2], xsum
+  static constexpr int kNumBars = 2 + 2 * kSlots + 10;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
-  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
-  static_assert(kAlloc <= 232448, "shared memory budget");
+  static constexpr int kAlloc = kBytes + 1024 <= 232448 ? kBytes + 1024 : 232448;
+  static_assert(kBytes <= 232448, "shared memory budget");
+  // Tensor-memory columns.
+  static constexpr uint32_t kColQ = 0;
+  static constexpr uint32_t kColS = 64;    // buffer b at kColS + 128 b
+  static constexpr uint32_t kColO = 320;
+  static constexpr uint32_t kColL = kColO + D;  // 16 columns: row sums of the 16-bit P
 };
 
 template <int D, bool BF16, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o_ptr,
-               float* __restrict__ lse_ptr, int Nq, int Nk, float scale_log2, int num_pairs) {
+               float* __restrict__ lse_ptr, int Nq, int Nk, float scale_log2) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
+  uint64_t* q_tmem = bars + 1;
+  uint64_t* kv_full = bars + 2;
   uint64_t* kv_empty = kv_full + L::kSlots;
   uint64_t* s_full = kv_empty + L::kSlots;
   uint64_t* p_full = s_full + 2;
-  uint64_t* o_full = p_full + 2;
-  uint64_t* mma_done = o_full + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* o_full = pv_done + 1;
+  uint64_t* mma_done = o_full + 1;
+  uint64_t* xmax_bar = mma_done + 1;  // [2], 256 arrivals each
+  uint64_t* xsum_bar = xmax_bar + 2;  // 256 arrivals
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  float* xchg = reinterpret_cast<float*>(smem + L::kXOff);                 // [2 parity][2 wg][128]
+  float* xsum = reinterpret_cast<float*>(smem + L::kXOff + L::kXBytes / 2);  // [2 sums][2 wg][128]
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int bh = blockIdx.x;
-  // Causal: the heaviest query-tile pairs are launched first.
-  const int pair = CAUSAL ? (num_pairs - 1 - static_cast<int>(blockIdx.y)) : static_cast<int>(blockIdx.y);
   const int nqt = Nq / kTile;
   const int nkt = Nk / kTile;
-  int n_kv[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int qt = 2 * pair + t;
-    n_kv[t] = qt < nqt ? (CAUSAL ? qt + 1 : nkt) : 0;
+  // Causal: the heaviest query tiles are launched first.
+  const int qt = CAUSAL ? (nqt - 1 - static_cast<int>(blockIdx.y)) : static_cast<int>(blockIdx.y);
+  const int n = CAUSAL ? qt + 1 : nkt;  // key tiles this query tile sees
+
+  // Refuse to run (and report) if alignment left too little shared memory.
+  if (static_cast<uint32_t>(smem - smem_raw) + L::kBytes > dynamic_smem_bytes()) {
+    if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusSmem);
+    return;
   }
-  const int nkv = n_kv[0] > n_kv[1] ? n_kv[0] : n_kv[1];
-  const int ntiles = n_kv[1] > 0 ? 2 : 1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_tmem, 256);
     for (int i = 0; i < L::kSlots; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
-      mbar_init(&o_full[t], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 256);
     }
+    mbar_init(pv_done, 1);
+    mbar_init(o_full, 1);
     mbar_init(mma_done, 1);
+    mbar_init(&xmax_bar[0], 256);
+    mbar_init(&xmax_bar[1], 256);
+    mbar_init(xsum_bar, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
+  }
+  if (warp == 3) {
+    const uint32_t one2 = BF16 ? 0x3F803F80u : 0x3C003C00u;  // two 16-bit ones
+    uint4* ones = reinterpret_cast<uint4*>(smem + L::kOnesOff);
+    for (int i = lane; i < L::kOnesBytes / 16; i += 32) ones[i] = make_uint4(one2, one2, one2, one2);
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -113,29 +157,27 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      const int qrow0 = bh * Nq + 2 * pair * kTile;
-      mbar_arrive_expect_tx(q_full, ntiles * L::kTileBytes);
-      for (int t = 0; t < ntiles; ++t)
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_2d(smem + L::kQOff + t * L::kTileBytes + c * L::kChunkBytes, &tm_q, q_full, c * 64,
-                      qrow0 + t * kTile);
+      mbar_arrive_expect_tx(q_full, L::kTileBytes);
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_2d(smem + L::kQOff + c * L::kChunkBytes, &tm_q, q_full, c * 64, bh * Nq + qt * kTile);
+      // Ring order: K_0, K_1, then V_j, K_{j+2} for j = 0, 1, ...
       const int krow0 = bh * Nk;
       int item = 0;
       bool ok = true;
-      for (int j = 0; j < nkv && ok; ++j) {
-        for (int which = 0; which < 2; ++which, ++item) {
-          const int slot = item % L::kSlots;
-          const uint32_t ph = (item / L::kSlots) & 1;
-          if (!mbar_wait(&kv_empty[slot], ph ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
-          uint8_t* dst = smem + L::kRingOff + slot * L::kTileBytes;
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_load_2d(dst + c * L::kChunkBytes, which ? &tm_v : &tm_k, &kv_full[slot], c * 64,
-                        krow0 + j * kTile);
-        }
+      auto load = [&](const CUtensorMap* map, int tile) {
+        const int slot = item % L::kSlots;
+        if (!mbar_wait(&kv_empty[slot], ((item / L::kSlots) & 1) ^ 1, abort_flag)) return false;
+        mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
+        uint8_t* dst = smem + L::kRingOff + slot * L::kTileBytes;
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_2d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * 64, krow0 + tile * kTile);
+        ++item;
+        return true;
+      };
+      for (int j = 0; ok && j < 2 && j < n; ++j) ok = load(&tm_k, j);
+      for (int j = 0; ok && j < n; ++j) {
+        ok = load(&tm_v, j);
+        if (ok && j + 2 < n) ok = load(&tm_k, j + 2);
       }
       if (!ok) {
         // Let the copies already issued land before the CTA exits.
@@ -146,202 +188,235 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);
-      constexpr uint32_t kIdPV = idesc_f16(BF16, 128, D, false, true);
-      const uint32_t q_base = smem_u32(smem + L::kQOff);
-      const uint32_t ring_base = smem_u32(smem + L::kRingOff);
-      auto slot_addr = [&](int item) { return ring_base + (item % L::kSlots) * L::kTileBytes; };
-      auto slot_of = [&](int item) { return item % L::kSlots; };
-      auto ph_of = [&](int item) { return static_cast<uint32_t>((item / L::kSlots) & 1); };
-      // S_t = Q_t K^T: both operands K-major; a K step of 16 elements is 32
-      // bytes inside a 128-byte swizzle row, 4 steps per 64-column chunk.
-      auto issue_s = [&](int t, uint32_t k_addr) {
-        const uint32_t qa = q_base + t * L::kTileBytes;
+    // The whole warp runs the loop (descriptors stay warp-uniform); one
+    // elected lane issues each group of MMAs together with its commits.
+    constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // A = Q (TMEM), B = K K-major
+    constexpr uint32_t kIdPV = idesc_f16(BF16, 128, D, false, true);    // A = P (TMEM), B = V MN-major
+    const uint32_t ring_base = smem_u32(smem + L::kRingOff);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    int item = 0;  // ring position, same order as the producer
+    auto wait_slot = [&](uint32_t& addr) {
+      const int slot = item % L::kSlots;
+      addr = ring_base + slot * L::kTileBytes;
+      return wait_all(&kv_full[slot], (item / L::kSlots) & 1);
+    };
+    // S = Q K^T: A = Q in TMEM (8 columns per K step of 16), B = K K-major
+    // (a K step is 32 bytes inside a 128-byte swizzle row).
+    auto issue_s = [&](int b, uint32_t k_addr) {
+      const uint64_t kd = sdesc_sw128(k_addr, 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-          mma_ss(tmem + t * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), kIdS,
-                 ks > 0 ? 1u : 0u);
-        }
-      };
-      // O_t += P_t V: P from TMEM (two 16-bit values per column, 8 columns per
-      // K step), V MN-major: a K step of 16 keys is 16 rows of 128 bytes.
-      auto issue_pv = [&](int t, uint32_t v_addr, bool acc) {
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
+        mma_ts(tmem + L::kColS + 128 * b, tmem + L::kColQ + 8 * ks, kd + (off >> 4), kIdS, ks > 0 ? 1u : 0u);
+      }
+    };
+    // O += P V: P in the buffer's TMEM columns (key step ks of 16 keys sits
+    // at 64 (ks / 4) + 8 (ks % 4)), V MN-major (16 rows of 128 bytes); then
+    // L += P 1 against the ones tile (two 256-byte core matrices per step).
+    constexpr uint32_t kIdL = idesc_f16(BF16, 128, 16, false, false);
+    const uint64_t ones_d = sdesc_noswz(smem_u32(smem + L::kOnesOff), 256, 128);
+    auto issue_pv = [&](int b, uint32_t v_addr, bool acc) {
+      const uint64_t vd = sdesc_sw128(v_addr, L::kChunkBytes, 1024);
 #pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_ts(tmem + 256 + t * D, tmem + t * 128 + ks * 8,
-                 sdesc_sw128(v_addr + ks * 2048, L::kChunkBytes, 1024), kIdPV, (acc || ks > 0) ? 1u : 0u);
-      };
+      for (int ks = 0; ks < kTile / 16; ++ks)
+        mma_ts(tmem + L::kColO, tmem + L::kColS + 128 * b + 64 * (ks >> 2) + 8 * (ks & 3), vd + 128 * ks, kIdPV,
+               (acc || ks > 0) ? 1u : 0u);
+#pragma unroll
+      for (int ks = 0; ks < kTile / 16; ++ks)
+        mma_ts(tmem + L::kColL, tmem + L::kColS + 128 * b + 64 * (ks >> 2) + 8 * (ks & 3), ones_d + 32 * ks, kIdL,
+               (acc || ks > 0) ? 1u : 0u);
+    };
 
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      if (ok && nkv > 0) {
-        ok = mbar_wait(&kv_full[slot_of(0)], ph_of(0), abort_flag);
-        if (ok) {
-          tc_fence_after();
-          for (int t = 0; t < 2; ++t)
-            if (n_kv[t] > 0) {
-              issue_s(t, slot_addr(0));
-              mma_commit(&s_full[t]);
-            }
-          mma_commit(&kv_empty[slot_of(0)]);
-        }
+    bool ok = wait_all(q_tmem, 0);
+    for (int j = 0; ok && j < 2 && j < n; ++j) {
+      uint32_t ka;
+      if (!(ok = wait_slot(ka))) break;
+      tc_fence_after();
+      if (elect_one()) {
+        issue_s(j, ka);
+        mma_commit(&s_full[j]);
+        mma_commit(&kv_empty[item % L::kSlots]);
       }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int vi = 2 * j + 1;  // ring item of V_j
-        const int ki = 2 * j + 2;  // ring item of K_{j+1}
-        if (!mbar_wait(&kv_full[slot_of(vi)], ph_of(vi), abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        bool k_next = false;
-        for (int t = 0; t < 2; ++t) {
-          if (j < n_kv[t]) {
-            if (!mbar_wait(&p_full[t], j & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_pv(t, slot_addr(vi), j > 0);
-            if (j == n_kv[t] - 1) mma_commit(&o_full[t]);
-          }
-          if (j + 1 < n_kv[t]) {
-            if (!k_next) {
-              if (!mbar_wait(&kv_full[slot_of(ki)], ph_of(ki), abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              k_next = true;
-            }
-            issue_s(t, slot_addr(ki));
-            mma_commit(&s_full[t]);
-          }
-        }
-        if (!ok) break;
-        mma_commit(&kv_empty[slot_of(vi)]);
-        if (k_next) mma_commit(&kv_empty[slot_of(ki)]);
-      }
-      // Every MMA issued above has completed once mma_done flips.
-      mma_commit(mma_done);
-      mbar_drain(mma_done, 0);
+      __syncwarp();
+      ++item;
     }
+    for (int j = 0; ok && j < n; ++j) {
+      const int b = j & 1;
+      uint32_t va;
+      if (!(ok = wait_slot(va))) break;
+      if (!(ok = wait_all(&p_full[b], (j >> 1) & 1))) break;
+      tc_fence_after();
+      if (elect_one()) {
+        issue_pv(b, va, j > 0);
+        mma_commit(pv_done);
+        mma_commit(&kv_empty[item % L::kSlots]);
+        if (j == n - 1) mma_commit(o_full);
+      }
+      __syncwarp();
+      ++item;
+      if (j + 2 < n) {
+        uint32_t ka;
+        if (!(ok = wait_slot(ka))) break;
+        tc_fence_after();
+        if (elect_one()) {
+          issue_s(b, ka);  // P(j) in this buffer was consumed by PV(j) above
+          mma_commit(&s_full[b]);
+          mma_commit(&kv_empty[item % L::kSlots]);
+        }
+        __syncwarp();
+        ++item;
+      }
+    }
+    if (elect_one()) mma_commit(mma_done);
+    __syncwarp();
+    mbar_drain(mma_done, 0);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 4) >> 2;     // query tile of this warpgroup
-    const int wq = warp & 3;           // 32-lane TMEM slice of this warp
-    const int row = wq * 32 + lane;    // query row within the tile
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t s_tm = tmem + lane_off + t * 128;
-    const uint32_t o_tm = tmem + lane_off + 256 + t * D;
-    const int n = n_kv[t];
-    const int qt = 2 * pair + t;
-    float m_run = -INFINITY;  // running max of the scores, log2 units (stale by < 8)
-    float l_run = 0.f;        // running sum of exp2(score - m_run)
-    float l_o = 0.f;          // the same sum over the 16-bit rounded terms
+    const int h = (warp - 4) >> 2;   // key columns [64h, 64h + 64) of each tile
+    const int wq = warp & 3;         // 32-lane TMEM slice of this warp
+    const int row = wq * 32 + lane;  // query row within the tile
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+
+    // Q -> TMEM: this thread copies its row's half of the head dimension
+    // (16-byte units of the 128-byte swizzled tile) as 16-bit pairs.
+    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag));
+    if (ok) {
+      constexpr int kUnits = D / 16;  // 16-byte units in half a row
+      const uint8_t* qrow = smem + L::kQOff + (D == 128 ? h * L::kChunkBytes : 0) + row * 128;
+      uint32_t qv[4 * kUnits];
+#pragma unroll
+      for (int u = 0; u < kUnits; ++u) {
+        const int unit = (D == 128 ? u : kUnits * h + u) ^ (row & 7);
+        const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + unit * 16);
+        qv[4 * u] = v4.x; qv[4 * u + 1] = v4.y; qv[4 * u + 2] = v4.z; qv[4 * u + 3] = v4.w;
+      }
+      if constexpr (D == 128) {
+        tmem_st32(t_row + L::kColQ + 32 * h, qv);
+      } else {
+        tmem_st16(t_row + L::kColQ + 16 * h, qv);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+    }
+    mbar_arrive(q_tmem);
+
     const bool pos_scale = scale_log2 > 0.f;
     const float cx = pos_scale ? scale_log2 : 1.f;
-    bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      ok = mbar_wait(&s_full[t], j & 1, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
+    float m_run = -INFINITY;  // running row max (log2 units; stale by < 8)
+    float l_run = 0.f;        // this warpgroup's part of sum exp2(score - m_run)
+    for (int j = 0; ok && j < n; ++j) {
+      const int b = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      // Scores of this row.  With a positive scale, the scale is folded into
-      // the exponent's FMA and the maximum is taken on the raw scores;
-      // otherwise the scores are scaled first.
-      float x[kTile];
+      const uint32_t s_col = t_row + L::kColS + 128 * b + 64 * h;
+      float x[64];
+      {
+        uint32_t r[64];
+        tmem_ld64(s_col, r);
 #pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(s_tm + c * 32, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(r[i]);
       }
       if (!pos_scale) {
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) x[c] *= scale_log2;
+        for (int c = 0; c < 64; ++c) x[c] *= scale_log2;
       }
       if (CAUSAL && j == qt) {
 #pragma unroll
-        for (int c = 0; c < kTile; ++c)
-          if (c > row) x[c] = -INFINITY;
+        for (int c = 0; c < 64; ++c)
+          if (64 * h + c > row) x[c] = -INFINITY;
       }
       float mp[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mp[i] = x[i];
 #pragma unroll
-      for (int c = 8; c < kTile; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
-      const float m_tile = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                                 fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * cx;
-      const float m_new = fmaxf(m_run, m_tile);
+      for (int c = 8; c < 64; c += 2) mp[(c >> 1) & 7] = max3f(mp[(c >> 1) & 7], x[c], x[c + 1]);
+      float mx = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+      // Row maximum over both halves of the key tile, exchanged through
+      // shared memory (double-buffered by tile parity: a warpgroup cannot
+      // rewrite a slot before the other has passed the next exchange, which
+      // it reaches only after reading the slot).
+      xchg[(b * 2 + h) * kTile + row] = mx;
+      mbar_arrive(&xmax_bar[b]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&xmax_bar[b], (j >> 1) & 1, abort_flag));
+      if (!ok) break;
+      mx = fmaxf(mx, xchg[(b * 2 + (h ^ 1)) * kTile + row]);
+      const float m_new = fmaxf(m_run, mx * cx);
       // Rescale O and the sums only when the maximum has grown by more than
-      // 2^8; otherwise keep the stale maximum (P stays below 256).
+      // 2^8; otherwise keep the stale maximum (P stays below 256).  Both
+      // warpgroups see the same m_run and m_new, so they decide alike.
       const bool need = (j > 0) && (m_new - m_run > 8.f);
       if (j == 0) m_run = m_new;
       if (__any_sync(0xffffffffu, need)) {
+        // O must hold PV(j-1) complete before it is rescaled.
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
         const float alpha = need ? ex2(m_run - m_new) : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t r[32];
-          tmem_ld32(o_tm + c * 32, r);
+          tmem_ld32(t_row + L::kColO + (D / 2) * h + 32 * c, r);
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(o_tm + c * 32, r);
+          tmem_st32(t_row + L::kColO + (D / 2) * h + 32 * c, r);
         }
+        if (h == 0) tmem_st1(t_row + L::kColL, __float_as_uint(__uint_as_float(tmem_ld1(t_row + L::kColL)) * alpha));
         if (need) {
           l_run *= alpha;
-          l_o *= alpha;
           m_run = m_new;
         }
       }
-      // l_run sums the fp32 probabilities (for LSE); l_o sums the rounded
-      // 16-bit probabilities that the P V product uses, so that O / l_o is a
-      // weighted mean of V rows with weights summing to one.
-      float su[4] = {0.f, 0.f, 0.f, 0.f}, sr[4] = {0.f, 0.f, 0.f, 0.f};
-      const float neg_m = -m_run;
+      // l_run sums the fp32 probabilities (for LSE); the tensor core sums
+      // the rounded 16-bit ones (L).  Arguments and sums as packed fp32x2.
+      float2 su[4];
 #pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) {
+      for (int i = 0; i < 4; ++i) su[i] = make_float2(0.f, 0.f);
+      const float2 cx2 = make_float2(cx, cx), negm2 = make_float2(-m_run, -m_run);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(x[c * 32 + 2 * i], cx, neg_m));
-          const float p1 = ex2(fmaf(x[c * 32 + 2 * i + 1], cx, neg_m));
-          pk[i] = pack2<BF16>(p0, p1);
-          const float2 pr = unpack2<BF16>(pk[i]);
-          su[i & 3] += p0 + p1;
-          sr[i & 3] += pr.x + pr.y;
+          const float2 a = fma2(make_float2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), cx2, negm2);
+          const float2 p = make_float2(ex2(a.x), ex2(a.y));
+          pk[i] = pack2<BF16>(p.x, p.y);
+          su[i & 3] = add2(su[i & 3], p);
         }
-        tmem_st16(s_tm + c * 16, pk);
+        tmem_st16(s_col + 16 * c, pk);
       }
-      l_run += (su[0] + su[1]) + (su[2] + su[3]);
-      l_o += (sr[0] + sr[1]) + (sr[2] + sr[3]);
+      const float2 su01 = add2(su[0], su[1]), su23 = add2(su[2], su[3]);
+      l_run += (su01.x + su01.y) + (su23.x + su23.y);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      mbar_arrive(&p_full[b]);
     }
+    // Epilogue: combine the two warpgroups' row sums, then each warpgroup
+    // writes its half of the head dimension of O.
+    xsum[h * kTile + row] = l_run;
+    mbar_arrive(xsum_bar);
+    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(xsum_bar, 0, abort_flag));
+    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort_flag));
     if (ok && n > 0) {
-      ok = mbar_wait(&o_full[t], 0, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok) {
-        tc_fence_after();
-        const float inv = 1.f / l_o;
-        const size_t grow = static_cast<size_t>(bh) * Nq + static_cast<size_t>(qt) * kTile + row;
-        uint4* dst = reinterpret_cast<uint4*>(o_ptr + grow * D);
+      tc_fence_after();
+      const float l_tot = l_run + xsum[(h ^ 1) * kTile + row];
+      const float inv = 1.f / __uint_as_float(tmem_ld1(t_row + L::kColL));
+      const size_t grow = static_cast<size_t>(bh) * Nq + static_cast<size_t>(qt) * kTile + row;
+      uint4* dst = reinterpret_cast<uint4*>(o_ptr + grow * D + (D / 2) * h);
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(o_tm + c * 32, r);
-          uint32_t pk[16];
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_row + L::kColO + (D / 2) * h + 32 * c, r);
+        uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
-        lse_ptr[grow] = (m_run + lg2(l_run)) * 0.69314718055994530942f;
+        for (int v = 0; v < 4; ++v) dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
+      if (h == 0) lse_ptr[grow] = (m_run + lg2(l_tot)) * 0.69314718055994530942f;
     }
   }
 
