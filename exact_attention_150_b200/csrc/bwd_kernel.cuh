@@ -231,87 +231,103 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // K-major x K-major
-      constexpr uint32_t kIdAcc = idesc_f16(BF16, 128, D, false, true);   // TMEM A x MN-major B
-      constexpr uint32_t kIdDK = idesc_f16(BF16, 128, D, false, true);    // K-major smem A x MN-major B
-      // dQ^T = K^T dS^T (M = d) or dQ = dS K (M = queries); both operands MN-major.
-      constexpr uint32_t kIdQ = kDqT ? idesc_f16(BF16, 128, 128, true, true) : idesc_f16(BF16, 128, 64, true, true);
-      const uint32_t k_addr = smem_u32(smem + L::kKOff);
-      const uint32_t v_addr = smem_u32(smem + L::kVOff);
-      const uint32_t ds_addr = smem_u32(smem + L::kDSOff);
-      auto stage_addr = [&](int it) {
-        return smem_u32(smem + L::kStageOff + (it % L::kStages) * 2 * L::kTileBytes);
-      };
-      // Packed 16-bit P^T / dS^T columns of K step ks (16 queries).
-      auto p_col = [](int ks) { return static_cast<uint32_t>(64 * (ks >> 2) + 8 * (ks & 3)); };
-      auto issue_st = [&](uint32_t q_addr) {
+    // The whole warp runs the loop (descriptors stay warp-uniform); one
+    // elected lane issues each group of MMAs together with its commits.
+    constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // K-major x K-major
+    constexpr uint32_t kIdAcc = idesc_f16(BF16, 128, D, false, true);   // K-major A x MN-major B
+    // dQ^T = K^T dS^T (M = d) or dQ = dS K (M = queries); both operands MN-major.
+    constexpr uint32_t kIdQ = kDqT ? idesc_f16(BF16, 128, 128, true, true) : idesc_f16(BF16, 128, 64, true, true);
+    const uint32_t k_addr = smem_u32(smem + L::kKOff);
+    const uint32_t v_addr = smem_u32(smem + L::kVOff);
+    const uint32_t ds_addr = smem_u32(smem + L::kDSOff);
+    // K-major SW128 operands step 32 bytes per K step inside a 128-byte row
+    // and 16 KB per 64-column chunk; MN-major ones step 16 rows (2048 bytes).
+    auto kmaj = [](int ks) { return static_cast<uint64_t>(((ks >> 2) * L::kChunkBytes + (ks & 3) * 32) >> 4); };
+    const uint64_t kd_k = sdesc_sw128(k_addr, 16, 1024), kd_v = sdesc_sw128(v_addr, 16, 1024);
+    const uint64_t kd_ds = sdesc_sw128(ds_addr, 16, 1024);
+    const uint64_t mn_k = sdesc_sw128(k_addr, L::kChunkBytes, 1024), mn_ds = sdesc_sw128(ds_addr, L::kChunkBytes, 1024);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    auto stage_addr = [&](int it) {
+      return smem_u32(smem + L::kStageOff + (it % L::kStages) * 2 * L::kTileBytes);
+    };
+    // Packed 16-bit P^T columns of K step ks (16 queries).
+    auto p_col = [](int ks) { return static_cast<uint32_t>(64 * (ks >> 2) + 8 * (ks & 3)); };
+    auto issue_st = [&](uint32_t q_addr) {
+      const uint64_t qd = sdesc_sw128(q_addr, 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-          mma_ss(tmem, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), kIdS,
-                 ks > 0 ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(kv_full, 0, abort_flag) && mbar_wait(&qd_full[0], 0, abort_flag);
-      if (ok && n_it > 0) {
-        tc_fence_after();
+      for (int ks = 0; ks < D / 16; ++ks) mma_ss(tmem, kd_k + kmaj(ks), qd + kmaj(ks), kIdS, ks > 0 ? 1u : 0u);
+    };
+    bool ok = wait_all(kv_full, 0) && wait_all(&qd_full[0], 0);
+    if (ok && n_it > 0) {
+      tc_fence_after();
+      if (elect_one()) {
         issue_st(stage_addr(0));
         mma_commit(s_full);
       }
-      for (int it = 0; ok && it < n_it; ++it) {
-        const uint32_t q_addr = stage_addr(it);
-        const uint32_t do_addr = q_addr + L::kTileBytes;
-        // dP^T overwrites the previous tile's dQ columns: wait for the drain.
-        if (it > 0 && !mbar_wait(dq_free, (it - 1) & 1, abort_flag)) break;
-        tc_fence_after();
+      __syncwarp();
+    }
+    for (int it = 0; ok && it < n_it; ++it) {
+      const uint32_t q_addr = stage_addr(it);
+      const uint32_t do_addr = q_addr + L::kTileBytes;
+      const uint64_t dod_k = sdesc_sw128(do_addr, 16, 1024);
+      const uint64_t dod_mn = sdesc_sw128(do_addr, L::kChunkBytes, 1024);
+      const uint64_t qd_mn = sdesc_sw128(q_addr, L::kChunkBytes, 1024);
+      // dP^T overwrites the previous tile's dQ columns: wait for the drain.
+      if (it > 0 && !(ok = wait_all(dq_free, (it - 1) & 1))) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-          mma_ss(tmem + kColDP, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024), kIdS,
-                 ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ss(tmem + kColDP, kd_v + kmaj(ks), dod_k + kmaj(ks), kIdS, ks > 0 ? 1u : 0u);
         mma_commit(dp_full);
-        if (!mbar_wait(p_full, it & 1, abort_flag)) break;
-        tc_fence_after();
+      }
+      __syncwarp();
+      if (!(ok = wait_all(p_full, it & 1))) break;
+      tc_fence_after();
+      if (elect_one()) {
         // dV += P^T dO: A from TMEM, B = dO MN-major (16 query rows per K step).
 #pragma unroll
         for (int ks = 0; ks < kBwdTile / 16; ++ks)
-          mma_ts(tmem + kColDV, tmem + p_col(ks), sdesc_sw128(do_addr + ks * 2048, L::kChunkBytes, 1024), kIdAcc,
-                 (it > 0 || ks > 0) ? 1u : 0u);
-        // The next tile's S^T only overwrites P^T, which dV (issued above)
-        // consumes first; issuing it now lets the softmax warps move on to
-        // the next P pass as soon as this tile's dS pass is done.
-        if (it + 1 < n_it) {
-          if (!mbar_wait(&qd_full[(it + 1) % L::kStages], ((it + 1) / L::kStages) & 1, abort_flag)) break;
-          tc_fence_after();
+          mma_ts(tmem + kColDV, tmem + p_col(ks), dod_mn + 128 * ks, kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+      // The next tile's S^T only overwrites P^T, which dV (issued above)
+      // consumes first; issuing it now lets the softmax warps move on to
+      // the next P pass as soon as this tile's dS pass is done.
+      if (it + 1 < n_it) {
+        if (!(ok = wait_all(&qd_full[(it + 1) % L::kStages], ((it + 1) / L::kStages) & 1))) break;
+        tc_fence_after();
+        if (elect_one()) {
           issue_st(stage_addr(it + 1));
           mma_commit(s_full);
         }
-        if (!mbar_wait(ds_full, it & 1, abort_flag)) break;
-        tc_fence_after();
-        // dK += dS^T Q: A = dS^T K-major in shared memory (16 queries = 32
-        // bytes per K step, 4 steps per 64-query chunk), B = Q MN-major.
+        __syncwarp();
+      }
+      if (!(ok = wait_all(ds_full, it & 1))) break;
+      tc_fence_after();
+      if (elect_one()) {
+        // dK += dS^T Q: A = dS^T K-major in shared memory, B = Q MN-major.
 #pragma unroll
         for (int ks = 0; ks < kBwdTile / 16; ++ks)
-          mma_ss(tmem + kColDK, sdesc_sw128(ds_addr + (ks >> 2) * L::kChunkBytes + (ks & 3) * 32, 16, 1024),
-                 sdesc_sw128(q_addr + ks * 2048, L::kChunkBytes, 1024), kIdDK, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(tmem + kColDK, kd_ds + kmaj(ks), qd_mn + 128 * ks, kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&qd_empty[it % L::kStages]);
         if (it == n_it - 1) mma_commit(acc_full);
 #pragma unroll
         for (int ks = 0; ks < kBwdTile / 16; ++ks) {
           if constexpr (kDqT)  // A = K^T (M = d), B = dS^T (N = queries)
-            mma_ss(tmem + kColDQ, sdesc_sw128(k_addr + ks * 2048, L::kChunkBytes, 1024),
-                   sdesc_sw128(ds_addr + ks * 2048, L::kChunkBytes, 1024), kIdQ, ks > 0 ? 1u : 0u);
+            mma_ss(tmem + kColDQ, mn_k + 128 * ks, mn_ds + 128 * ks, kIdQ, ks > 0 ? 1u : 0u);
           else  // A = dS (M = queries), B = K (N = d)
-            mma_ss(tmem + kColDQ, sdesc_sw128(ds_addr + ks * 2048, L::kChunkBytes, 1024),
-                   sdesc_sw128(k_addr + ks * 2048, L::kChunkBytes, 1024), kIdQ, ks > 0 ? 1u : 0u);
+            mma_ss(tmem + kColDQ, mn_ds + 128 * ks, mn_k + 128 * ks, kIdQ, ks > 0 ? 1u : 0u);
         }
         mma_commit(dq_full);
       }
-      mma_commit(mma_done);
-      mbar_drain(mma_done, 0);
+      __syncwarp();
     }
+    if (elect_one()) mma_commit(mma_done);
+    __syncwarp();
+    mbar_drain(mma_done, 0);
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ P and dS
     const int h = (warp - 4) >> 2;  // query columns [64h, 64h + 64)

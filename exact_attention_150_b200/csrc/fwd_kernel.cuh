@@ -381,7 +381,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float2 a = fma2(make_float2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), cx2, negm2);
-          const float2 p = make_float2(ex2(a.x), ex2(a.y));
+          // One pair in four on the FMA pipe: MUFU throughput bounds the
+          // exponentials otherwise.
+          const float2 p = ((i & 3) == 3) ? exp2_poly2(a) : make_float2(ex2(a.x), ex2(a.y));
           pk[i] = pack2<BF16>(p.x, p.y);
           su[i & 3] = add2(su[i & 3], p);
         }
