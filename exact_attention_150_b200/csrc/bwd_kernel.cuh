@@ -7,10 +7,10 @@
 //   bwd_pre_kernel    D_i = sum_c dO_ic O_ic, -log2(e) * LSE_i, and dQacc = 0
 //   bwd_main_kernel   one CTA per (key tile j, batch*head): K_j, V_j stay in
 //                     shared memory; for every query tile i that sees them
-//                       S^T  = K_j Q_i^T              (tcgen05, TMEM)
-//                       dP^T = V_j dO_i^T             (tcgen05, TMEM)
-//                       P^T  = exp2(S^T * scale*log2e - LSE_i*log2e)
-//                       dS^T = P^T * (dP^T - D_i)
+//                       S'^T  = K_j Q_i^T - LSE_i / scale   (tcgen05, TMEM)
+//                       dP'^T = V_j dO_i^T - D_i            (tcgen05, TMEM)
+//                       P^T   = exp2(S'^T * scale * log2e)
+//                       dS^T  = P^T * dP'^T
 //                       dV_j += P^T dO_i              (A = P^T from TMEM)
 //                       dK_j += dS^T Q_i              (A = dS^T from shared memory)
 //                       dQacc_i += scale * dS K_j     (fp32 atomics)
@@ -41,6 +41,13 @@
 //   dP^T, dV, S^T(next), dK, dQ
 // and the softmax warps go from this tile's dS pass straight to the next
 // tile's P pass while dK and dQ run on the tensor core.
+// The per-query terms -LSE_i / scale and -D_i enter through one extra K step
+// of 16 in the S^T and dP^T products: the A operand is a constant tile that
+// selects them ([1,1,0,...] or [0,0,1,1,0,...] in every key row) and the B
+// operand holds, per query row, each term as a 16-bit high part plus a
+// 16-bit remainder.  The softmax warps thus need no per-query data at all.
+// Warp 3 writes that B block for the next query tile while the current one
+// is in use (single buffer, released by the dP^T product).
 #pragma once
 
 #include "sm100.cuh"
@@ -59,12 +66,17 @@ struct BwdLayout {
   static constexpr int kStageOff = 2 * kTileBytes;  // stage s: Q at +s*2T, dO at +s*2T+T
   static constexpr int kDSOff = kStageOff + kStages * 2 * kTileBytes;
   static constexpr int kDSBytes = kBwdTile * kBwdTile * 2;
-  // Per stage: -log2(e) LSE and D of the stage's 128 query rows (512 B each).
-  static constexpr int kVecOff = kDSOff + kDSBytes;
-  static constexpr int kVecBytes = 2 * kBwdTile * 4;
-  static constexpr int kBarOff = kVecOff + kStages * kVecBytes;
-  // kv_full, qd_full[S], qd_empty[S], s_full, dp_full, p_full, ds_full, dq_full, dq_free, acc_full, mma_done
-  static constexpr int kNumBars = 1 + 2 * kStages + 8;
+  // Extra K step: A_ext = two unswizzled 8x16-byte core matrices per term
+  // (selector row, zeros), read with a zero row-group stride; B_ext = 128
+  // query rows x 16 bytes [s_hi, s_lo, d_hi, d_lo, 0, 0, 0, 0].
+  static constexpr int kAExtOff = kDSOff + kDSBytes;
+  static constexpr int kAExtBytes = 4 * 128;
+  static constexpr int kBExtOff = kAExtOff + kAExtBytes;
+  static constexpr int kBExtBytes = kBwdTile * 16;
+  static constexpr int kBarOff = kBExtOff + kBExtBytes;
+  // kv_full, qd_full[S], qd_empty[S], s_full, dp_full, p_full, ds_full, dq_full, dq_free, acc_full, mma_done,
+  // bext_full, bext_free
+  static constexpr int kNumBars = 1 + 2 * kStages + 10;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   // The tiles need a 1024-byte aligned base.  The dynamic shared window
@@ -147,6 +159,8 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* dq_free = s_full + 5;
   uint64_t* acc_full = s_full + 6;
   uint64_t* mma_done = s_full + 7;
+  uint64_t* bext_full = s_full + 8;  // warp 3 -> MMA: B_ext holds the current tile's terms
+  uint64_t* bext_free = s_full + 9;  // MMA -> warp 3: the dP^T product has read B_ext
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -178,12 +192,24 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(dq_free, 128);
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
+    mbar_init(bext_full, 32);
+    mbar_init(bext_free, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
+  }
+  if (warp == 3) {
+    // A_ext: [sel_s: rows of 1,1,0,..] [zeros] [sel_d: rows of 0,0,1,1,0,..] [zeros]
+    const uint32_t one = BF16 ? 0x3F80u : 0x3C00u;
+    uint32_t* a = reinterpret_cast<uint32_t*>(smem + L::kAExtOff);
+    for (int i = lane; i < L::kAExtBytes / 4; i += 32) {
+      const int cm = i / 32, w = i % 4;  // core matrix, 32-bit word within a 16-byte row
+      a[i] = (cm == 0 && w == 0) || (cm == 2 && w == 1) ? (one | (one << 16)) : 0u;
+    }
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -213,15 +239,12 @@ __global__ void __launch_bounds__(512, 1)
           break;
         }
         const int qrow = bh * Nq + (i0 + it) * kBwdTile;
-        mbar_arrive_expect_tx(&qd_full[s], 2 * L::kTileBytes + L::kVecBytes);
+        mbar_arrive_expect_tx(&qd_full[s], 2 * L::kTileBytes);
         uint8_t* qdst = smem + L::kStageOff + s * 2 * L::kTileBytes;
         for (int c = 0; c < D / 64; ++c) {
           tma_load_2d(qdst + c * L::kChunkBytes, &tm_q, &qd_full[s], c * 64, qrow);
           tma_load_2d(qdst + L::kTileBytes + c * L::kChunkBytes, &tm_do, &qd_full[s], c * 64, qrow);
         }
-        uint8_t* vdst = smem + L::kVecOff + s * L::kVecBytes;
-        bulk_load(vdst, nlse2 + qrow, kBwdTile * 4, &qd_full[s]);
-        bulk_load(vdst + kBwdTile * 4, dvec + qrow, kBwdTile * 4, &qd_full[s]);
       }
       if (!ok) {
         mbar_drain(kv_full, 0);
@@ -254,12 +277,21 @@ __global__ void __launch_bounds__(512, 1)
     };
     // Packed 16-bit P^T columns of K step ks (16 queries).
     auto p_col = [](int ks) { return static_cast<uint32_t>(64 * (ks >> 2) + 8 * (ks & 3)); };
+    // Extra K step: A_ext selects a term (zero row-group stride: one core
+    // matrix serves all 128 rows), B_ext holds it per query row.
+    const uint64_t ext_s = sdesc_noswz(smem_u32(smem + L::kAExtOff), 128, 0);
+    const uint64_t ext_d = sdesc_noswz(smem_u32(smem + L::kAExtOff + 256), 128, 0);
+    const uint64_t ext_b = sdesc_noswz(smem_u32(smem + L::kBExtOff), 0, 128);
+    const bool zero_scale = scale == 0.f;  // then S' is the LSE term alone
     auto issue_st = [&](uint32_t q_addr) {
       const uint64_t qd = sdesc_sw128(q_addr, 16, 1024);
+      if (!zero_scale) {
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) mma_ss(tmem, kd_k + kmaj(ks), qd + kmaj(ks), kIdS, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < D / 16; ++ks) mma_ss(tmem, kd_k + kmaj(ks), qd + kmaj(ks), kIdS, ks > 0 ? 1u : 0u);
+      }
+      mma_ss(tmem, ext_s, ext_b, kIdS, zero_scale ? 0u : 1u);
     };
-    bool ok = wait_all(kv_full, 0) && wait_all(&qd_full[0], 0);
+    bool ok = wait_all(kv_full, 0) && wait_all(&qd_full[0], 0) && wait_all(bext_full, 0);
     if (ok && n_it > 0) {
       tc_fence_after();
       if (elect_one()) {
@@ -281,7 +313,9 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
           mma_ss(tmem + kColDP, kd_v + kmaj(ks), dod_k + kmaj(ks), kIdS, ks > 0 ? 1u : 0u);
+        mma_ss(tmem + kColDP, ext_d, ext_b, kIdS, 1u);
         mma_commit(dp_full);
+        mma_commit(bext_free);  // S^T and dP^T of this tile have read B_ext
       }
       __syncwarp();
       if (!(ok = wait_all(p_full, it & 1))) break;
@@ -298,6 +332,7 @@ __global__ void __launch_bounds__(512, 1)
       // the next P pass as soon as this tile's dS pass is done.
       if (it + 1 < n_it) {
         if (!(ok = wait_all(&qd_full[(it + 1) % L::kStages], ((it + 1) / L::kStages) & 1))) break;
+        if (!(ok = wait_all(bext_full, (it + 1) & 1))) break;
         tc_fence_after();
         if (elect_one()) {
           issue_st(stage_addr(it + 1));
@@ -328,11 +363,38 @@ __global__ void __launch_bounds__(512, 1)
     if (elect_one()) mma_commit(mma_done);
     __syncwarp();
     mbar_drain(mma_done, 0);
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ B_ext writer
+    // Row q of B_ext: [s_hi, s_lo, d_hi, d_lo, 0, 0, 0, 0] with s = -LSE_q /
+    // scale (-log2(e) LSE_q when scale == 0) and d = -D_q, each split into a
+    // 16-bit value and the 16-bit rounding of its remainder.
+    const float inv_c = scale == 0.f ? 1.f : 1.f / scale_log2;  // nlse2 = -log2(e) LSE
+    uint4* bext = reinterpret_cast<uint4*>(smem + L::kBExtOff);
+    auto split = [](float v) {
+      const float hi = unpack2<BF16>(pack2<BF16>(v, 0.f)).x;
+      return pack2<BF16>(hi, v - hi);
+    };
+    for (int it = 0; it < n_it; ++it) {
+      const size_t vbase = static_cast<size_t>(bh) * Nq + static_cast<size_t>(i0 + it) * kBwdTile;
+      float sv[4], dv4[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        sv[k] = nlse2[vbase + lane + 32 * k] * inv_c;
+        dv4[k] = -dvec[vbase + lane + 32 * k];
+      }
+      if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(bext_free, (it - 1) & 1, abort_flag))) break;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) bext[lane + 32 * k] = make_uint4(split(sv[k]), split(dv4[k]), 0u, 0u);
+      fence_proxy_async_smem();
+      mbar_arrive(bext_full);
+    }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ P and dS
     const int h = (warp - 4) >> 2;  // query columns [64h, 64h + 64)
     const int wq = warp & 3;
     const int r = wq * 32 + lane;   // key row within tile j = TMEM lane
+    const float cs = scale == 0.f ? 1.f : scale_log2;  // S' is in units of 1 / scale
+    const float2 cs2 = make_float2(cs, cs);
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     uint8_t* ds_row = smem + L::kDSOff + h * L::kChunkBytes + r * 128;
     for (int it = 0; it < n_it; ++it) {
@@ -340,29 +402,20 @@ __global__ void __launch_bounds__(512, 1)
       const bool diag = CAUSAL && i == j;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag))) break;
       tc_fence_after();
-      // -log2(e) LSE and D of this warpgroup's 64 queries, staged by the
-      // producer with the stage's Q and dO.  Each lane reads two of each
-      // (coalesced); the inner loops broadcast them with warp shuffles, so
-      // no shared-memory access sits on their critical path.
-      const float* vec = reinterpret_cast<const float*>(smem + L::kVecOff + (it % L::kStages) * L::kVecBytes);
-      const float nl_lo = vec[64 * h + lane], nl_hi = vec[64 * h + 32 + lane];
-      const float dd_lo = vec[kBwdTile + 64 * h + lane], dd_hi = vec[kBwdTile + 64 * h + 32 + lane];
-      // P pass: P^T = exp2(S^T * scale * log2e - LSE * log2e), packed 16-bit.
+      // P pass: P^T = exp2(S'^T * scale * log2e), packed 16-bit.
       uint32_t ppk[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t sr[32];
         tmem_ld32(t_row + 64 * h + 32 * c, sr);
-        const float nl_src = c ? nl_hi : nl_lo;
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
             const int x = 16 * g + e;
-            const float n0 = __shfl_sync(0xffffffffu, nl_src, x);
-            const float n1 = __shfl_sync(0xffffffffu, nl_src, x + 1);
-            float p0 = ex2(fmaf(__uint_as_float(sr[x]), scale_log2, n0));
-            float p1 = ex2(fmaf(__uint_as_float(sr[x + 1]), scale_log2, n1));
+            const float2 a = mul2(make_float2(__uint_as_float(sr[x]), __uint_as_float(sr[x + 1])), cs2);
+            float p0 = ex2(a.x);
+            float p1 = ex2(a.y);
             if (diag) {  // key r is visible to query q iff r <= q
               const int q = 64 * h + 32 * c + x;
               if (r > q) p0 = 0.f;
@@ -384,7 +437,7 @@ __global__ void __launch_bounds__(512, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
-      // dS pass: dS^T = P^T * (dP^T - D), packed 16-bit into the 128-byte-
+      // dS pass: dS^T = P^T * dP'^T, packed 16-bit into the 128-byte-
       // swizzled shared tile (row r, 64 queries per 16 KB chunk).
       if (!__all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag))) break;
       tc_fence_after();
@@ -392,17 +445,15 @@ __global__ void __launch_bounds__(512, 1)
       for (int c = 0; c < 2; ++c) {
         uint32_t pr[32];
         tmem_ld32(t_row + kColDP + 64 * h + 32 * c, pr);
-        const float dd_src = c ? dd_hi : dd_lo;
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           uint32_t dpk[8];
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
             const int x = 16 * g + e;
-            const float d0 = __shfl_sync(0xffffffffu, dd_src, x);
-            const float d1 = __shfl_sync(0xffffffffu, dd_src, x + 1);
-            const float2 p = unpack2<BF16>(ppk[16 * c + x / 2]);
-            dpk[e / 2] = pack2<BF16>(p.x * (__uint_as_float(pr[x]) - d0), p.y * (__uint_as_float(pr[x + 1]) - d1));
+            const float2 d = mul2(unpack2<BF16>(ppk[16 * c + x / 2]),
+                                  make_float2(__uint_as_float(pr[x]), __uint_as_float(pr[x + 1])));
+            dpk[e / 2] = pack2<BF16>(d.x, d.y);
           }
 #pragma unroll
           for (int v = 0; v < 2; ++v) {
