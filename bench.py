@@ -40,9 +40,9 @@ METRIC = "attention fwd/bwd TFLOP/s on 1 B200 and fraction of dense BF16/FP16 te
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 # dram__bytes_read.sum + dram__bytes_write.sum of one bwd_main_kernel launch
-# (bf16, causal, d=128, B=1) from the one-pass ncu launch list summarised in
-# profiles/launches_long_ctx_N16384.md, keyed by (N, H).  Only valid for the
-# kernel version it was taken on: reset it to None when the kernel changes.
+# (bf16, causal, d=128, B=1), measured by a one-pass ncu capture of this
+# bench's full-size command and keyed by (N, H).  Only valid for the kernel
+# version it was taken on: reset it to None when the kernel changes.
 BWD_MAIN_TRAFFIC = {(16384, 16): 1982788352.0 + 1019262720.0}
 
 
