@@ -32,35 +32,45 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D view [rows][d] of a contiguous 16-bit tensor, read in boxes of 64
-// columns (128 bytes) x 128 rows with the 128-byte swizzle the MMA
-// descriptors expect.
-bool make_map(CUtensorMap* map, const void* base, long long rows, int d, bool bf16) {
+// 3D view [B*H][N][d] of a contiguous 16-bit tensor, read in boxes of 64
+// columns (128 bytes) x 128 rows of one (b, h) slice with the 128-byte
+// swizzle the MMA descriptors expect.  Rows past N read as zeros, so a
+// ragged last tile never touches the next slice.
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTile)};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTile), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
+int tiles(int n) { return (n + kTile - 1) / kTile; }
+
+// Rows after the dQ accumulator that a ragged last query tile of the last
+// (b, h) slice reduces into.  The main kernel reduces all 128 rows of every
+// query tile without a per-row test; the rows past Nq carry exact zeros
+// (their probabilities are masked and their dO rows read as zeros), so in
+// other slices they land harmlessly on the next slice's first rows, and in
+// the last slice they land here.
+long long pad_rows(int Nq) { return static_cast<long long>(tiles(Nq)) * kTile - Nq; }
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-attn_status check_common(int B, int H, int Nq, int Nk, int d, int causal, attn_dtype dtype) {
-  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+// Sizes may be zero (an empty problem); they may not be negative.
+attn_status check_common(int B, int H, int Nq, int Nk, int d, attn_dtype dtype) {
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d < 0) return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_FP16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (Nq % kTile != 0 || Nk % kTile != 0) return ATTN_ERR_UNSUPPORTED;
-  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
   const long long bh = static_cast<long long>(B) * H;
-  // TMA row coordinates and grid dimensions are 32-bit.
-  if (bh > 0x7fffffffLL || bh * Nq > 0x7fffffffLL || bh * Nk > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  if (Nq / kTile > 65535 || Nk / kTile > 65535) return ATTN_ERR_UNSUPPORTED;
+  // Grid x and TMA coordinates are 32-bit; grid y is 16-bit.
+  if (bh > 0x7fffffffLL || tiles(Nq) > 65535 || tiles(Nk) > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (bh * Nq > (1LL << 40) || bh * Nk > (1LL << 40)) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 
@@ -75,7 +85,7 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   using L = attn::FwdLayout<D>;
   auto kern = attn::fwd_kernel<D, BF16, CAUSAL>;
   if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
-  dim3 grid(BH, Nq / kTile);
+  dim3 grid(BH, tiles(Nq));
   kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, Nq, Nk, scale_log2);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -87,7 +97,7 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   using L = attn::BwdLayout<D>;
   const long long qrows = static_cast<long long>(BH) * Nq;
   float* dqacc = ws;
-  float* dvec = ws + qrows * D;
+  float* dvec = ws + (qrows + pad_rows(Nq)) * D;
   float* nlse2 = dvec + qrows;
 
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_PREPROCESS) {
@@ -100,7 +110,7 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_MAIN) {
     auto kern = attn::bwd_main_kernel<D, BF16, CAUSAL>;
     if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
-    dim3 grid(BH, Nk / kTile);
+    dim3 grid(BH, tiles(Nk));
     kern<<<grid, 512, L::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, dqacc, static_cast<uint16_t*>(dk),
                                        static_cast<uint16_t*>(dv), Nq, Nk, scale, scale * 1.4426950408889634f);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -175,17 +185,17 @@ extern "C" {
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
                      int d, float scale, int causal, attn_dtype dtype, void* stream) {
+  const attn_status cs = check_common(B, H, Nq, Nk, d, dtype);
+  if (cs != ATTN_OK) return cs;
+  if (B == 0 || H == 0 || Nq == 0) return ATTN_OK;  // no query rows: nothing to write
+  if (Nk == 0) return ATTN_ERR_INVALID_ARG;         // a softmax over no keys is undefined
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return ATTN_ERR_INVALID_ARG;
-  const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
-  if (cs != ATTN_OK) return cs;
   const bool bf16 = dtype == ATTN_BF16;
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, static_cast<long long>(BH) * Nq, d, bf16) ||
-      !make_map(&mk, k, static_cast<long long>(BH) * Nk, d, bf16) ||
-      !make_map(&mv, v, static_cast<long long>(BH) * Nk, d, bf16))
+  if (!make_map(&mq, q, BH, Nq, d, bf16) || !make_map(&mk, k, BH, Nk, d, bf16) || !make_map(&mv, v, BH, Nk, d, bf16))
     return ATTN_ERR_CUDA;
   const float sl2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -197,9 +207,10 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
-  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return 0;
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return 0;  // empty problems need none
   const unsigned long long rows = static_cast<unsigned long long>(B) * H * Nq;
-  const unsigned long long floats = rows * (static_cast<unsigned long long>(d) + 2);
+  const unsigned long long floats =
+      (rows + static_cast<unsigned long long>(pad_rows(Nq))) * static_cast<unsigned long long>(d) + 2 * rows;
   if (floats > (~0ull) / 4) return 0;
   return static_cast<size_t>(floats * 4);
 }
@@ -215,19 +226,29 @@ attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const vo
                            const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq,
                            int Nk, int d, float scale, int causal, attn_dtype dtype, int phase, void* stream) {
   if (phase < ATTN_BWD_ALL || phase > ATTN_BWD_CONVERT) return ATTN_ERR_INVALID_ARG;
+  const attn_status cs = check_common(B, H, Nq, Nk, d, dtype);
+  if (cs != ATTN_OK) return cs;
+  if (B == 0 || H == 0) return ATTN_OK;
+  if (Nk == 0) return Nq == 0 ? ATTN_OK : ATTN_ERR_INVALID_ARG;
+  cudaStream_t st0 = static_cast<cudaStream_t>(stream);
+  if (Nq == 0) {
+    // No query rows: dK = dV = 0 (written by the main phase), dQ is empty.
+    if (!dk || !dv) return ATTN_ERR_INVALID_ARG;
+    if (phase != ATTN_BWD_ALL && phase != ATTN_BWD_MAIN) return ATTN_OK;
+    const size_t bytes = static_cast<size_t>(B) * H * Nk * d * 2;
+    if (cudaMemsetAsync(dk, 0, bytes, st0) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, st0) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    return ATTN_OK;
+  }
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
   for (const void* p : ptrs)
     if (!aligned16(p)) return ATTN_ERR_INVALID_ARG;
-  const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
-  if (cs != ATTN_OK) return cs;
   const bool bf16 = dtype == ATTN_BF16;
   const int BH = B * H;
   CUtensorMap mq, mk, mv, mdo;
-  if (!make_map(&mq, q, static_cast<long long>(BH) * Nq, d, bf16) ||
-      !make_map(&mk, k, static_cast<long long>(BH) * Nk, d, bf16) ||
-      !make_map(&mv, v, static_cast<long long>(BH) * Nk, d, bf16) ||
-      !make_map(&mdo, dout, static_cast<long long>(BH) * Nq, d, bf16))
+  if (!make_map(&mq, q, BH, Nq, d, bf16) || !make_map(&mk, k, BH, Nk, d, bf16) ||
+      !make_map(&mv, v, BH, Nk, d, bf16) || !make_map(&mdo, dout, BH, Nq, d, bf16))
     return ATTN_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
@@ -241,13 +262,15 @@ attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const vo
 attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                              const void* dout, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d,
                              float scale, int causal, attn_dtype dtype, void* stream) {
-  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
-  const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
+  const attn_status cs = check_common(B, H, Nq, Nk, d, dtype);
   if (cs != ATTN_OK) return cs;
   if (attn_bwd_workspace_bytes(B, H, Nq, Nk, d) > kNoAllocScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
-  const attn_status ss = scratch_for_current_device(&scratch);
-  if (ss != ATTN_OK) return ss;
+  if (B > 0 && H > 0 && Nq > 0 && Nk > 0) {
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+    const attn_status ss = scratch_for_current_device(&scratch);
+    if (ss != ATTN_OK) return ss;
+  }
   // The preprocess kernel rewrites every byte of the scratch that the main
   // kernel reads (it zeroes the dQ accumulator), so the previous call's
   // contents never leak into this one.

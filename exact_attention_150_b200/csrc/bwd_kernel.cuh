@@ -168,9 +168,22 @@ __global__ void __launch_bounds__(512, 1)
   const int lane = threadIdx.x % 32;
   const int bh = blockIdx.x;
   const int j = blockIdx.y;  // key tile; causal: small j has the most work and launches first
-  const int nqt = Nq / kBwdTile;
+  const int nqt = (Nq + kBwdTile - 1) / kBwdTile;  // the last tiles may be ragged
   const int i0 = CAUSAL ? j : 0;
   const int n_it = nqt - i0;
+  const int kv_valid = Nk - j * kBwdTile < kBwdTile ? Nk - j * kBwdTile : kBwdTile;  // key rows of this tile
+
+  if (n_it <= 0) {
+    // Causal with more keys than queries: no query sees these keys, so
+    // their gradients are zero.
+    const int n16 = kv_valid * D / 8;
+    const size_t base = (static_cast<size_t>(bh) * Nk + static_cast<size_t>(j) * kBwdTile) * D / 8;
+    for (int e = threadIdx.x; e < n16; e += blockDim.x) {
+      reinterpret_cast<uint4*>(dk_ptr)[base + e] = make_uint4(0u, 0u, 0u, 0u);
+      reinterpret_cast<uint4*>(dv_ptr)[base + e] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    return;
+  }
 
   // Refuse to run (and report) if alignment left too little shared memory.
   if (static_cast<uint32_t>(smem - smem_raw) + L::kBytes > dynamic_smem_bytes()) {
@@ -223,11 +236,10 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      const int krow = bh * Nk + j * kBwdTile;
       mbar_arrive_expect_tx(kv_full, 2 * L::kTileBytes);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_2d(smem + L::kKOff + c * L::kChunkBytes, &tm_k, kv_full, c * 64, krow);
-        tma_load_2d(smem + L::kVOff + c * L::kChunkBytes, &tm_v, kv_full, c * 64, krow);
+        tma_load_3d(smem + L::kKOff + c * L::kChunkBytes, &tm_k, kv_full, c * 64, j * kBwdTile, bh);
+        tma_load_3d(smem + L::kVOff + c * L::kChunkBytes, &tm_v, kv_full, c * 64, j * kBwdTile, bh);
       }
       int it = 0;
       bool ok = true;
@@ -238,12 +250,12 @@ __global__ void __launch_bounds__(512, 1)
           ok = false;
           break;
         }
-        const int qrow = bh * Nq + (i0 + it) * kBwdTile;
+        const int qrow = (i0 + it) * kBwdTile;
         mbar_arrive_expect_tx(&qd_full[s], 2 * L::kTileBytes);
         uint8_t* qdst = smem + L::kStageOff + s * 2 * L::kTileBytes;
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_2d(qdst + c * L::kChunkBytes, &tm_q, &qd_full[s], c * 64, qrow);
-          tma_load_2d(qdst + L::kTileBytes + c * L::kChunkBytes, &tm_do, &qd_full[s], c * 64, qrow);
+          tma_load_3d(qdst + c * L::kChunkBytes, &tm_q, &qd_full[s], c * 64, qrow, bh);
+          tma_load_3d(qdst + L::kTileBytes + c * L::kChunkBytes, &tm_do, &qd_full[s], c * 64, qrow, bh);
         }
       }
       if (!ok) {
@@ -376,11 +388,13 @@ __global__ void __launch_bounds__(512, 1)
     };
     for (int it = 0; it < n_it; ++it) {
       const size_t vbase = static_cast<size_t>(bh) * Nq + static_cast<size_t>(i0 + it) * kBwdTile;
+      const int q_valid = Nq - (i0 + it) * kBwdTile;
       float sv[4], dv4[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        sv[k] = nlse2[vbase + lane + 32 * k] * inv_c;
-        dv4[k] = -dvec[vbase + lane + 32 * k];
+        const bool in = lane + 32 * k < q_valid;  // rows past Nq: zeros (their P is masked)
+        sv[k] = in ? nlse2[vbase + lane + 32 * k] * inv_c : 0.f;
+        dv4[k] = in ? -dvec[vbase + lane + 32 * k] : 0.f;
       }
       if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(bext_free, (it - 1) & 1, abort_flag))) break;
 #pragma unroll
@@ -400,6 +414,15 @@ __global__ void __launch_bounds__(512, 1)
     for (int it = 0; it < n_it; ++it) {
       const int i = i0 + it;
       const bool diag = CAUSAL && i == j;
+      // Key row r sees query columns [lo, hi) of this tile: lo = r on the
+      // diagonal tile (key after query is masked), hi = the queries before
+      // Nq, and none at all if the key is past Nk.  P is zeroed outside.
+      const int q_valid = Nq - i * kBwdTile;
+      const bool masked = diag || kv_valid < kBwdTile || q_valid < kBwdTile;
+      const int lo = diag ? r : 0;
+      const int hi = r < kv_valid ? (q_valid < kBwdTile ? q_valid : kBwdTile) : 0;
+      const uint32_t span = hi > lo ? static_cast<uint32_t>(hi - lo) : 0u;
+      const int q_base = 64 * h - lo;  // column q tests (q - lo) < span, unsigned
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag))) break;
       tc_fence_after();
       // P pass: P^T = exp2(S'^T * scale * log2e), packed 16-bit.
@@ -416,10 +439,10 @@ __global__ void __launch_bounds__(512, 1)
             const float2 a = mul2(make_float2(__uint_as_float(sr[x]), __uint_as_float(sr[x + 1])), cs2);
             float p0 = ex2(a.x);
             float p1 = ex2(a.y);
-            if (diag) {  // key r is visible to query q iff r <= q
-              const int q = 64 * h + 32 * c + x;
-              if (r > q) p0 = 0.f;
-              if (r > q + 1) p1 = 0.f;
+            if (masked) {
+              const int q = q_base + 32 * c + x;
+              if (static_cast<uint32_t>(q) >= span) p0 = 0.f;
+              if (static_cast<uint32_t>(q + 1) >= span) p1 = 0.f;
             }
             ppk[16 * c + x / 2] = pack2<BF16>(p0, p1);
           }
@@ -482,7 +505,9 @@ __global__ void __launch_bounds__(512, 1)
         // Thread = head-dim index d; a warp's reduction covers 32 consecutive
         // d of one query row (128 contiguous bytes).
         // All 128 columns are read before the columns are released, so the
-        // next dP^T product does not wait for the reductions.
+        // next dP^T product does not wait for the reductions.  Query rows
+        // past Nq in a ragged tile hold exact zeros (masked P) and are
+        // reduced like the others; the host pads the accumulator for them.
         float* base = dqacc + qrow0 * D + row;
         uint32_t va[32], vb[32], vc[32], vd[32];
         tmem_ld32(t_row + kColDQ, va);
@@ -492,7 +517,8 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_before();
         mbar_arrive(dq_free);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) atomicAdd(base + static_cast<size_t>(q) * D, __uint_as_float(va[q]) * scale);
+        for (int q = 0; q < 32; ++q)
+          atomicAdd(base + static_cast<size_t>(q) * D, __uint_as_float(va[q]) * scale);
 #pragma unroll
         for (int q = 0; q < 32; ++q)
           atomicAdd(base + static_cast<size_t>(32 + q) * D, __uint_as_float(vb[q]) * scale);
@@ -527,6 +553,7 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
         // dK / dV: M = keys, so the TMEM lane is the key row.
         const size_t grow = static_cast<size_t>(bh) * Nk + static_cast<size_t>(j) * kBwdTile + row;
+        const bool live = row < kv_valid;  // padding rows of a ragged key tile are not stored
         uint4* dvd = reinterpret_cast<uint4*>(dv_ptr + grow * D);
         uint4* dkd = reinterpret_cast<uint4*>(dk_ptr + grow * D);
 #pragma unroll 1
@@ -535,14 +562,18 @@ __global__ void __launch_bounds__(512, 1)
           tmem_ld32(t_row + kColDV + c * 32, rv);
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack2<BF16>(__uint_as_float(rv[2 * e]), __uint_as_float(rv[2 * e + 1]));
+          if (live) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dvd[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int v = 0; v < 4; ++v) dvd[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
           tmem_ld32(t_row + kColDK + c * 32, rv);
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             pk[e] = pack2<BF16>(__uint_as_float(rv[2 * e]) * scale, __uint_as_float(rv[2 * e + 1]) * scale);
+          if (live) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dkd[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int v = 0; v < 4; ++v) dkd[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
         }
       }
     }

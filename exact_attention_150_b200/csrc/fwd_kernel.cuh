@@ -104,11 +104,12 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int bh = blockIdx.x;
-  const int nqt = Nq / kTile;
-  const int nkt = Nk / kTile;
+  const int nqt = (Nq + kTile - 1) / kTile;  // the last tiles may be ragged
+  const int nkt = (Nk + kTile - 1) / kTile;
   // Causal: the heaviest query tiles are launched first.
   const int qt = CAUSAL ? (nqt - 1 - static_cast<int>(blockIdx.y)) : static_cast<int>(blockIdx.y);
-  const int n = CAUSAL ? qt + 1 : nkt;  // key tiles this query tile sees
+  // Key tiles this query tile sees (top-left causal: key <= query).
+  const int n = CAUSAL ? (qt + 1 < nkt ? qt + 1 : nkt) : nkt;
 
   // Refuse to run (and report) if alignment left too little shared memory.
   if (static_cast<uint32_t>(smem - smem_raw) + L::kBytes > dynamic_smem_bytes()) {
@@ -159,9 +160,8 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(q_full, L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
-        tma_load_2d(smem + L::kQOff + c * L::kChunkBytes, &tm_q, q_full, c * 64, bh * Nq + qt * kTile);
+        tma_load_3d(smem + L::kQOff + c * L::kChunkBytes, &tm_q, q_full, c * 64, qt * kTile, bh);
       // Ring order: K_0, K_1, then V_j, K_{j+2} for j = 0, 1, ...
-      const int krow0 = bh * Nk;
       int item = 0;
       bool ok = true;
       auto load = [&](const CUtensorMap* map, int tile) {
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
         uint8_t* dst = smem + L::kRingOff + slot * L::kTileBytes;
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_2d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * 64, krow0 + tile * kTile);
+          tma_load_3d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * 64, tile * kTile, bh);
         ++item;
         return true;
       };
@@ -323,10 +323,15 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 64; ++c) x[c] *= scale_log2;
       }
-      if (CAUSAL && j == qt) {
+      // Mask keys past Nk (ragged last tile) and, on the diagonal tile,
+      // keys after this query (the tiles start at the same offset).
+      const int kv_valid = Nk - j * kTile;
+      if ((CAUSAL && j == qt) || kv_valid < kTile) {
+        int lim = kv_valid - 1;
+        if (CAUSAL && j == qt && row < lim) lim = row;
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if (64 * h + c > row) x[c] = -INFINITY;
+          if (64 * h + c > lim) x[c] = -INFINITY;
       }
       float mp[8];
 #pragma unroll
@@ -405,6 +410,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const float l_tot = l_run + xsum[(h ^ 1) * kTile + row];
       const float inv = 1.f / __uint_as_float(tmem_ld1(t_row + L::kColL));
+      const bool live = qt * kTile + row < Nq;  // padding rows of a ragged tile are not stored
       const size_t grow = static_cast<size_t>(bh) * Nq + static_cast<size_t>(qt) * kTile + row;
       uint4* dst = reinterpret_cast<uint4*>(o_ptr + grow * D + (D / 2) * h);
 #pragma unroll 1
@@ -415,10 +421,12 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           pk[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+        if (live) {
 #pragma unroll
-        for (int v = 0; v < 4; ++v) dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int v = 0; v < 4; ++v) dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
       }
-      if (h == 0) lse_ptr[grow] = (m_run + lg2(l_tot)) * 0.69314718055994530942f;
+      if (h == 0 && live) lse_ptr[grow] = (m_run + lg2(l_tot)) * 0.69314718055994530942f;
     }
   }
 

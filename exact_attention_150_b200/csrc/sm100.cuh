@@ -132,6 +132,16 @@ __device__ __forceinline__ uint32_t dynamic_smem_bytes() {
   return v;
 }
 
+// 3D tiled load of box (x, y, z) of `map`; rows of y past the extent of the
+// map are zero-filled.  x must be a multiple of 8 elements (16 bytes).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (tcgen05).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

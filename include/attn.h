@@ -26,15 +26,26 @@
  *   call only enqueues work on it and returns without synchronising.
  * Mask.  causal != 0 applies the top-left causal mask: query row i attends to
  *   key row j iff j <= i.  (The pages name a causal mask but not its
- *   alignment when Nq != Nk; top-left is the reading taken.)
+ *   alignment when Nq != Nk; top-left is the reading taken.  With Nq > Nk the
+ *   query rows past Nk see every key; with Nq < Nk the keys past Nq are seen
+ *   by no query, and their dK, dV are zero.)
  * LSE.  lse[b][h][i] = ln sum_j exp(scale * q_i . k_j) over the unmasked j:
  *   the natural-log row log-sum-exp of the scaled scores, in fp32.
- * Supported shapes.  d in {64, 128}; Nq and Nk multiples of 128; for causal,
- *   Nq == Nk.  Other shapes return ATTN_ERR_UNSUPPORTED.
+ * Supported shapes.  d in {64, 128}; any Nq, Nk >= 0 (the kernels work in
+ *   tiles of 128 rows and mask a ragged last tile); causal with any Nq, Nk.
+ *   The tile counts ceil(Nq / 128) and ceil(Nk / 128) must not exceed 65535
+ *   and B*H must fit in an int; other shapes return ATTN_ERR_UNSUPPORTED.
+ * Empty problems.  B, H, Nq or Nk may be 0.  A call with no query rows
+ *   (B*H*Nq == 0) is valid and does nothing, except that attn_bwd then writes
+ *   dK = dV = 0 (their rows exist but no query reaches them).  Nq > 0 with
+ *   Nk == 0 asks for a softmax over no keys, which is undefined, and returns
+ *   ATTN_ERR_INVALID_ARG.  Pointers of an empty tensor are not read and may
+ *   be NULL.
  * Errors.  Arguments are validated on the host before anything is enqueued:
- *   a NULL pointer, a non-positive size or a pointer that is not 16-byte
- *   aligned returns ATTN_ERR_INVALID_ARG; an unsupported shape or dtype returns
- *   ATTN_ERR_UNSUPPORTED; a failed launch returns ATTN_ERR_CUDA.  Nothing is
+ *   a negative size, a NULL pointer or a pointer that is not 16-byte aligned
+ *   (of a non-empty tensor) returns ATTN_ERR_INVALID_ARG; an unsupported shape
+ *   or dtype returns ATTN_ERR_UNSUPPORTED; a failed launch returns
+ *   ATTN_ERR_CUDA.  Nothing is
  *   written to any output when a call returns an error.  There is no fallback
  *   to another implementation.  Kernels never trap: a wait inside a kernel
  *   that exceeds its time limit makes the kernel record ATTN_ERR_TIMEOUT in a
@@ -71,8 +82,8 @@ typedef enum { ATTN_FP16 = 0, ATTN_BF16 = 1 } attn_dtype;
  *   q, k, v   inputs, read only.
  *   o         output [B][H][Nq][d], 16-bit.
  *   lse       output [B][H][Nq], float.
- *   B, H      batch and head count (> 0).
- *   Nq, Nk    query and key sequence lengths (> 0).
+ *   B, H      batch and head count (>= 0).
+ *   Nq, Nk    query and key sequence lengths (>= 0; see Empty problems).
  *   d         head dimension.
  *   scale     multiplier of Q K^T; the pages use 1/sqrt(d).
  */
@@ -82,9 +93,11 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
 
 /*
  * Size in bytes of the device workspace attn_bwd needs: an fp32 dQ
- * accumulator [B][H][Nq][d], then the fp32 row term D [B][H][Nq], then the
- * fp32 row term -log2(e) * LSE [B][H][Nq].  Returns 0 if a size is
- * non-positive or the total overflows size_t.
+ * accumulator [B][H][Nq][d] followed by (128 - Nq % 128) % 128 rows of d
+ * floats of padding (a ragged last query tile reduces its masked rows, which
+ * are exact zeros, into them), then the fp32 row term D [B][H][Nq], then the
+ * fp32 row term -log2(e) * LSE [B][H][Nq].  Returns 0 for an empty problem
+ * (any size 0), a negative size, or a total that overflows size_t.
  */
 size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d);
 
@@ -141,8 +154,8 @@ attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const vo
  * holds it until the process exits), and the caller still passes every input
  * and output.
  *   Limit.  Problems whose attn_bwd_workspace_bytes() exceeds
- *           attn_bwd_noalloc_max_scratch_bytes() (72 MiB; e.g. B*H*Nq up
- *           to 145,187 rows at d = 128) return ATTN_ERR_SCRATCH_LIMIT
+ *           attn_bwd_noalloc_max_scratch_bytes() (72 MiB; at d = 128 about
+ *           145,000 query rows B*H*Nq) return ATTN_ERR_SCRATCH_LIMIT
  *           before any work is enqueued.
  *   Set-up. The first call on each device looks up the array's device
  *           address (cudaGetSymbolAddress) with that device current; make

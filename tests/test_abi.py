@@ -78,14 +78,29 @@ def test_fwd_misaligned_pointer(lib):
 
 
 @pytest.mark.parametrize("field", ["B", "H", "Nq", "Nk", "d"])
-@pytest.mark.parametrize("value", [0, -128])
-def test_non_positive_sizes(lib, field, value):
-    assert _fwd(**{field: value}) == native.ATTN_ERR_INVALID_ARG
-    assert _bwd(**{field: value}) == native.ATTN_ERR_INVALID_ARG
+def test_negative_sizes(lib, field):
+    assert _fwd(**{field: -128}) == native.ATTN_ERR_INVALID_ARG
+    assert _bwd(**{field: -128}) == native.ATTN_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("kw", [dict(d=96), dict(d=256), dict(d=32), dict(Nq=200), dict(Nk=130),
-                                dict(Nq=128, Nk=256, causal=1), dict(dtype=2), dict(dtype=-1)])
+@pytest.mark.parametrize("field", ["B", "H", "Nq"])
+def test_empty_problem_is_a_no_op(lib, field):
+    """No query rows (or no batch/heads): nothing to write, so success without
+    touching any pointer or the device."""
+    nulls = dict(q=None, k=None, v=None, o=None, lse=None)
+    assert _fwd(**{field: 0}, **nulls) == native.ATTN_OK
+    if field != "Nq":  # Nq == 0 with keys still writes dK = dV = 0 (a device memset)
+        assert _bwd(**{field: 0}, **nulls, dout=None, dq=None, dk=None, dv=None, workspace=None) == native.ATTN_OK
+
+
+def test_no_keys_is_invalid(lib):
+    assert _fwd(Nk=0) == native.ATTN_ERR_INVALID_ARG
+    assert _bwd(Nk=0) == native.ATTN_ERR_INVALID_ARG
+    assert _bwd(Nk=0, Nq=0) == native.ATTN_OK
+
+
+@pytest.mark.parametrize("kw", [dict(d=96), dict(d=256), dict(d=32), dict(d=0), dict(dtype=2), dict(dtype=-1),
+                                dict(Nq=65535 * 128 + 1), dict(Nk=65535 * 128 + 1)])
 def test_unsupported_shapes(lib, kw):
     assert _fwd(**kw) == native.ATTN_ERR_UNSUPPORTED
     assert _bwd(**kw) == native.ATTN_ERR_UNSUPPORTED
@@ -96,6 +111,9 @@ def test_workspace_size(lib):
     assert native.attn_bwd_workspace_bytes(1, 16, 16384, 16384, 128) == 4 * 16 * 16384 * 130
     assert native.attn_bwd_workspace_bytes(0, 1, 128, 128, 64) == 0
     assert native.attn_bwd_workspace_bytes(1, 1, -1, 128, 64) == 0
+    # A ragged last query tile pads the dQ accumulator to a whole tile.
+    assert native.attn_bwd_workspace_bytes(2, 3, 300, 77, 64) == 4 * ((6 * 300 + 84) * 64 + 2 * 6 * 300)
+    assert native.attn_bwd_workspace_bytes(1, 1, 1, 1, 128) == 4 * (128 * 128 + 2)
 
 
 def test_tensor_wrapper_rejects_cpu_tensors(lib):
@@ -129,3 +147,5 @@ def test_bwd_phase_validates_like_bwd(lib):
     assert native.attn_bwd_phase(**args) == native.ATTN_ERR_UNSUPPORTED
     args.update(d=64, dq=None)
     assert native.attn_bwd_phase(**args) == native.ATTN_ERR_INVALID_ARG
+    args.update(B=0)
+    assert native.attn_bwd_phase(**args) == native.ATTN_OK

@@ -65,6 +65,34 @@ def test_backward_nq_ne_nk(nq, nk):
     check_grads_all_slices(q, k, v, do, False, 0.125, f"Nq{nq} Nk{nk}")
 
 
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n", [1, 5, 100, 129, 300])
+def test_backward_ragged(dtype, d, causal, n):
+    q, k, v, do = draw(1, 2, n, n, d, dtype, seed=400 + n + d, with_grad=True)
+    check_grads_all_slices(q, k, v, do, causal, 1.0 / math.sqrt(d), f"ragged N{n} d{d} {dtype} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("nq,nk", [(100, 300), (300, 100), (1, 257), (257, 1), (640, 200)])
+def test_backward_ragged_nq_ne_nk(causal, nq, nk):
+    """Includes key tiles no query sees (causal, Nk > Nq): their dK, dV are 0."""
+    q, k, v, do = draw(1, 2, nq, nk, 64, torch.float16, seed=31 + nq + nk, with_grad=True)
+    check_grads_all_slices(q, k, v, do, causal, 0.125, f"Nq{nq} Nk{nk} causal={causal}")
+
+
+def test_backward_no_queries_gives_zero_dk_dv():
+    q = torch.zeros(1, 2, 0, 64, dtype=torch.float16, device=DEV)
+    k = torch.randn(1, 2, 130, 64, device=DEV).half()
+    lse = torch.zeros(1, 2, 0, device=DEV)
+    dk = torch.full_like(k, 7.0)
+    dv = torch.full_like(k, 7.0)
+    native.backward(q, k, k, q, lse, q, dk=dk, dv=dv, workspace=torch.empty(0, dtype=torch.uint8, device=DEV))
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dk) == 0 and torch.count_nonzero(dv) == 0
+
+
 def test_backward_scale_zero_gives_zero_dq_dk():
     q, k, v, do = draw(1, 2, 256, 256, 64, torch.bfloat16, seed=22, with_grad=True)
     _, _, dq, dk, dv = run_fwd_bwd(q, k, v, do, True, 0.0)

@@ -86,13 +86,42 @@ def test_forward_constant_v_and_first_causal_row():
     np.testing.assert_allclose(lse[:, :, 0].double().numpy(), want.numpy(), atol=1e-4)
 
 
-def test_forward_unsupported_shapes_raise():
-    q = torch.zeros(1, 1, 200, 64, dtype=torch.float16, device=DEV)
-    with pytest.raises(native.AttnError):
-        native.forward(q, q, q)
+def test_forward_unsupported_head_dim_raises():
     q = torch.zeros(1, 1, 128, 96, dtype=torch.float16, device=DEV)
     with pytest.raises(native.AttnError):
         native.forward(q, q, q)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n", [1, 5, 100, 129, 300, 777])
+def test_forward_ragged(dtype, d, causal, n):
+    """Lengths that are not multiples of the 128-row tile: the last tile is
+    zero-filled by the tensor map, its padding keys are masked and its
+    padding query rows are not stored."""
+    q, k, v = draw(1, 3, n, n, d, dtype, seed=300 + n + d)
+    check_all_slices(q, k, v, causal, 1.0 / math.sqrt(d), f"ragged N{n} d{d} {dtype} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("nq,nk", [(100, 300), (300, 100), (129, 1), (1, 257), (640, 200)])
+def test_forward_ragged_nq_ne_nk(causal, nq, nk):
+    """Top-left causal with Nq != Nk: query i sees keys j <= i."""
+    q, k, v = draw(2, 2, nq, nk, 128, torch.bfloat16, seed=17 + nq + nk)
+    check_all_slices(q, k, v, causal, 1.0 / math.sqrt(128), f"Nq{nq} Nk{nk} causal={causal}")
+
+
+def test_forward_empty_problems():
+    for shape_q, shape_k in (((0, 2, 128, 64), (0, 2, 128, 64)), ((1, 2, 0, 64), (1, 2, 64, 64))):
+        q = torch.zeros(shape_q, dtype=torch.bfloat16, device=DEV)
+        k = torch.zeros(shape_k, dtype=torch.bfloat16, device=DEV)
+        o, lse = native.forward(q, k, k)
+        assert o.numel() == 0 and lse.numel() == 0
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16, device=DEV)
+    k = torch.zeros(1, 1, 0, 64, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(native.AttnError):
+        native.forward(q, k, k)
 
 
 # ---------------------------------------------------------- named workloads
