@@ -23,7 +23,7 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")
 
 def _expr(s: str) -> float:
     """Evaluate a golden expression: numbers, + - * / and log()."""
-    return float(eval(s, {"__builtins__": {}}, {"log": math.log, "Fraction": Fraction}))
+    return float(eval(s, {"__builtins__": {}}, {"log": math.log, "Fraction": Fraction, "inf": math.inf}))
 
 
 def _mat(rows) -> np.ndarray:
@@ -44,7 +44,8 @@ def _close(a, b, tol):
     b = np.asarray(b, dtype=np.float64)
     if a.shape != b.shape:
         return False
-    return bool(np.all(np.abs(a - b) <= tol * (1.0 + np.abs(b))))
+    with np.errstate(invalid="ignore"):
+        return bool(np.all((a == b) | (np.abs(a - b) <= tol * (1.0 + np.abs(b)))))
 
 
 def forward_pin_failures(fwd) -> list[str]:
@@ -56,8 +57,12 @@ def forward_pin_failures(fwd) -> list[str]:
     for case in g["forward"]:
         q, k, v = _mat(case["q"]), _mat(case["k"]), _mat(case["v"])
         s = _expr(case["scale"])
-        for mode, causal in (("noncausal", False), ("causal", True)):
-            o, lse, _ = fwd(q, k, v, s, causal)
+        # bottom-right: the causal diagonal ends at the last key (offset Nk - Nq).
+        for mode, causal, off in (("noncausal", False, 0), ("causal", True, 0),
+                                  ("bottom_right", True, k.shape[0] - q.shape[0])):
+            if mode not in case:
+                continue
+            o, lse, _ = fwd(q, k, v, s, causal, off)
             if not _close(o, _mat(case[mode]["o"]), 1e-12):
                 fails.append(f"golden {case['name']} {mode} O")
             want_lse = np.array([_expr(x) for x in case[mode]["lse"]])
@@ -109,6 +114,17 @@ def forward_pin_failures(fwd) -> list[str]:
     o, lse, _ = fwd(q, k, v, 1.3, False)
     if not _close(o, np.broadcast_to(v, o.shape), 1e-12):
         fails.append("single key")
+
+    # Rows that see no key (causal with a negative offset -m): O = 0,
+    # LSE = -inf, P = 0; the other rows are the problem without them.
+    m = 3
+    q, k, v = r.standard_normal((1, 2, 8, 3)), r.standard_normal((1, 2, 5, 3)), r.standard_normal((1, 2, 5, 4))
+    o, lse, p = fwd(q, k, v, 0.8, True, -m)
+    if np.any(o[..., :m, :] != 0) or np.any(lse[..., :m] != -np.inf) or np.any(p[..., :m, :] != 0):
+        fails.append("rows that see no key")
+    o2, lse2, _ = fwd(q[..., m:, :], k, v, 0.8, True, 0)
+    if not _close(o[..., m:, :], o2, 1e-12) or not _close(lse[..., m:], lse2, 1e-12):
+        fails.append("rows after those that see no key")
 
     # Permutation equivariance.
     q, k, v = r.standard_normal((2, 3, 8, 4)), r.standard_normal((2, 3, 8, 4)), r.standard_normal((2, 3, 8, 4))
@@ -167,7 +183,7 @@ def backward_pin_failures(bwd, fwd) -> list[str]:
     g = golden_cases()
     for case in g["backward"]:
         q, k, v, do = (_mat(case[x]) for x in ("q", "k", "v", "do"))
-        dq, dk, dv = bwd(q, k, v, do, _expr(case["scale"]), case["causal"])
+        dq, dk, dv = bwd(q, k, v, do, _expr(case["scale"]), case["causal"], case.get("q_offset", 0))
         for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
             if not _close(got, _mat(case[name]), 1e-12):
                 fails.append(f"golden {case['name']} {name}")
@@ -183,6 +199,17 @@ def backward_pin_failures(bwd, fwd) -> list[str]:
                 err = np.max(np.abs(a - b)) / max(1.0, np.max(np.abs(b)))
                 if not (err <= 1e-6):
                     fails.append(f"finite differences {name} n={n} d={d} causal={causal}")
+
+    # Rows that see no key add nothing: with offset -m, dQ of the first m
+    # rows is 0 and the rest equals the problem without those rows.
+    m = 2
+    q, do = r.standard_normal((1, 2, 7, 3)), r.standard_normal((1, 2, 7, 4))
+    k, v = r.standard_normal((1, 2, 4, 3)), r.standard_normal((1, 2, 4, 4))
+    dq, dk, dv = bwd(q, k, v, do, 0.9, True, -m)
+    dq2, dk2, dv2 = bwd(q[..., m:, :], k, v, do[..., m:, :], 0.9, True, 0)
+    if np.any(dq[..., :m, :] != 0) or not _close(dq[..., m:, :], dq2, 1e-12) or not _close(dk, dk2, 1e-12) \
+            or not _close(dv, dv2, 1e-12):
+        fails.append("backward rows that see no key")
 
     # Identities: sum over keys of dK is 0 (rows of dS sum to 0); sum over
     # keys of dV equals sum over queries of dO (columns of P^T sum to 1);

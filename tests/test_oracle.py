@@ -90,6 +90,11 @@ def _fwd_strict_mask(q, k, v, scale, causal, q_offset=0):
     return oracle.forward(q, k, v, scale, causal, q_offset)
 
 
+def _fwd_offset_sign(q, k, v, scale, causal, q_offset=0):
+    # diagonal shifted the wrong way (query i sees keys j <= i - offset)
+    return oracle.forward(q, k, v, scale, causal, -q_offset)
+
+
 def _fwd_lse_base2(q, k, v, scale, causal, q_offset=0):
     o, lse, p = oracle.forward(q, k, v, scale, causal, q_offset)
     return o, lse / np.log(2.0), p
@@ -114,10 +119,14 @@ def _fwd_swapped_qk(q, k, v, scale, causal, q_offset=0):
     if causal:
         nq, nk = s.shape[-2:]
         s = np.where(np.arange(nk)[None, :] > (q_offset + np.arange(nq))[:, None], -np.inf, s)
-    m = np.max(s, -1, keepdims=True)
+    # rows that see no key: empty softmax, O = 0, LSE = log 0
+    live = np.isfinite(s).any(-1, keepdims=True)
+    m = np.where(live, np.max(s, -1, keepdims=True), 0.0)
     e = np.exp(s - m)
-    p = e / e.sum(-1, keepdims=True)
-    return np.matmul(p, np.asarray(v, dtype=np.float64)), (m + np.log(e.sum(-1, keepdims=True)))[..., 0], p
+    tot = np.where(live, e.sum(-1, keepdims=True), 1.0)
+    p = e / tot
+    lse = np.where(live, m + np.log(tot), -np.inf)[..., 0]
+    return np.matmul(p, np.asarray(v, dtype=np.float64)), lse, p
 
 
 def _bwd_sign(q, k, v, do, scale, causal, q_offset=0):
@@ -145,7 +154,7 @@ def _bwd_dv_untransposed(q, k, v, do, scale, causal, q_offset=0):
     return dq, dk, p @ np.asarray(do, dtype=np.float64)
 
 
-@pytest.mark.parametrize("mutant", [_fwd_no_scale, _fwd_strict_mask, _fwd_lse_base2,
+@pytest.mark.parametrize("mutant", [_fwd_no_scale, _fwd_strict_mask, _fwd_offset_sign, _fwd_lse_base2,
                                     _fwd_reversed_v, _fwd_column_softmax])
 def test_planted_forward_mistakes_are_caught(mutant):
     try:
