@@ -63,8 +63,10 @@ long long pad_rows(int Nq) { return static_cast<long long>(tiles(Nq)) * kTile - 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Sizes may be zero (an empty problem); they may not be negative.
-attn_status check_common(int B, int H, int Nq, int Nk, int d, attn_dtype dtype) {
+attn_status check_common(int B, int H, int Nq, int Nk, int d, int causal, attn_dtype dtype) {
   if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d < 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != ATTN_CAUSAL_NONE && causal != ATTN_CAUSAL_TOP_LEFT && causal != ATTN_CAUSAL_BOTTOM_RIGHT)
+    return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_FP16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   const long long bh = static_cast<long long>(B) * H;
@@ -81,19 +83,19 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 template <int D, bool BF16, bool CAUSAL>
 attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse,
-                       int BH, int Nq, int Nk, float scale_log2, cudaStream_t st) {
+                       int BH, int Nq, int Nk, int off, float scale_log2, cudaStream_t st) {
   using L = attn::FwdLayout<D>;
   auto kern = attn::fwd_kernel<D, BF16, CAUSAL>;
   if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
   dim3 grid(BH, tiles(Nq));
-  kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, Nq, Nk, scale_log2);
+  kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, Nq, Nk, off, scale_log2);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <int D, bool BF16, bool CAUSAL>
 attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                        const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv, float* ws,
-                       int BH, int Nq, int Nk, float scale, int phase, cudaStream_t st) {
+                       int BH, int Nq, int Nk, int off, float scale, int phase, cudaStream_t st) {
   using L = attn::BwdLayout<D>;
   const long long qrows = static_cast<long long>(BH) * Nq;
   float* dqacc = ws;
@@ -112,7 +114,7 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
     dim3 grid(BH, tiles(Nk));
     kern<<<grid, 512, L::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, dqacc, static_cast<uint16_t*>(dk),
-                                       static_cast<uint16_t*>(dv), Nq, Nk, scale, scale * 1.4426950408889634f);
+                                       static_cast<uint16_t*>(dv), Nq, Nk, off, scale, scale * 1.4426950408889634f);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_CONVERT) {
@@ -126,11 +128,15 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   return ATTN_OK;
 }
 
+// Diagonal offset of the causal mask: query i sees key k iff k <= i + off.
+int causal_offset(int causal, int Nq, int Nk) { return causal == ATTN_CAUSAL_BOTTOM_RIGHT ? Nk - Nq : 0; }
+
 template <int D, bool BF16>
 attn_status dispatch_fwd_causal(int causal, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                 void* o, float* lse, int BH, int Nq, int Nk, float sl2, cudaStream_t st) {
-  return causal ? launch_fwd<D, BF16, true>(mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st)
-                : launch_fwd<D, BF16, false>(mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st);
+  const int off = causal_offset(causal, Nq, Nk);
+  return causal ? launch_fwd<D, BF16, true>(mq, mk, mv, o, lse, BH, Nq, Nk, off, sl2, st)
+                : launch_fwd<D, BF16, false>(mq, mk, mv, o, lse, BH, Nq, Nk, off, sl2, st);
 }
 
 template <int D, bool BF16>
@@ -138,9 +144,11 @@ attn_status dispatch_bwd_causal(int causal, const CUtensorMap& mq, const CUtenso
                                 const CUtensorMap& mdo, const void* o, const void* dout, const float* lse, void* dq,
                                 void* dk, void* dv, float* ws, int BH, int Nq, int Nk, float scale, int phase,
                                 cudaStream_t st) {
+  const int off = causal_offset(causal, Nq, Nk);
   return causal
-             ? launch_bwd<D, BF16, true>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st)
-             : launch_bwd<D, BF16, false>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st);
+             ? launch_bwd<D, BF16, true>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, off, scale, phase, st)
+             : launch_bwd<D, BF16, false>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, off, scale, phase,
+                                          st);
 }
 
 }  // namespace
@@ -185,7 +193,7 @@ extern "C" {
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
                      int d, float scale, int causal, attn_dtype dtype, void* stream) {
-  const attn_status cs = check_common(B, H, Nq, Nk, d, dtype);
+  const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
   if (B == 0 || H == 0 || Nq == 0) return ATTN_OK;  // no query rows: nothing to write
   if (Nk == 0) return ATTN_ERR_INVALID_ARG;         // a softmax over no keys is undefined
@@ -226,7 +234,7 @@ attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const vo
                            const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq,
                            int Nk, int d, float scale, int causal, attn_dtype dtype, int phase, void* stream) {
   if (phase < ATTN_BWD_ALL || phase > ATTN_BWD_CONVERT) return ATTN_ERR_INVALID_ARG;
-  const attn_status cs = check_common(B, H, Nq, Nk, d, dtype);
+  const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
   if (B == 0 || H == 0) return ATTN_OK;
   if (Nk == 0) return Nq == 0 ? ATTN_OK : ATTN_ERR_INVALID_ARG;
@@ -262,7 +270,7 @@ attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const vo
 attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                              const void* dout, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d,
                              float scale, int causal, attn_dtype dtype, void* stream) {
-  const attn_status cs = check_common(B, H, Nq, Nk, d, dtype);
+  const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
   if (attn_bwd_workspace_bytes(B, H, Nq, Nk, d) > kNoAllocScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;

@@ -118,7 +118,9 @@ __global__ void __launch_bounds__(256)
   for (int m = kTpr / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
   if (row < rows && seg == 0) {
     dvec[row] = acc;
-    nlse2[row] = -lse[row] * 1.4426950408889634074f;
+    // A row that sees no key (LSE = -inf) has every P masked; a finite
+    // stand-in keeps the extra MMA K step free of inf - inf.
+    nlse2[row] = lse[row] == -INFINITY ? 0.f : -lse[row] * 1.4426950408889634074f;
   }
 }
 
@@ -139,8 +141,8 @@ __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const float* __restrict__ dvec, const float* __restrict__ nlse2, float* __restrict__ dqacc,
-                    uint16_t* __restrict__ dk_ptr, uint16_t* __restrict__ dv_ptr, int Nq, int Nk, float scale,
-                    float scale_log2) {
+                    uint16_t* __restrict__ dk_ptr, uint16_t* __restrict__ dv_ptr, int Nq, int Nk, int off,
+                    float scale, float scale_log2) {
   using L = BwdLayout<D>;
   constexpr bool kDqT = (D == 128);  // dQ formed transposed (see above)
   constexpr uint32_t kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 256 + D;
@@ -169,7 +171,11 @@ __global__ void __launch_bounds__(512, 1)
   const int bh = blockIdx.x;
   const int j = blockIdx.y;  // key tile; causal: small j has the most work and launches first
   const int nqt = (Nq + kBwdTile - 1) / kBwdTile;  // the last tiles may be ragged
-  const int i0 = CAUSAL ? j : 0;
+  // Causal: query q sees key k iff k <= q + off (off = 0 top-left,
+  // Nk - Nq bottom-right); the first query tile that sees key j * 128 is
+  // the one holding query j * 128 - off.
+  const int first_q = j * kBwdTile - off;
+  const int i0 = CAUSAL ? (first_q > 0 ? first_q / kBwdTile : 0) : 0;
   const int n_it = nqt - i0;
   const int kv_valid = Nk - j * kBwdTile < kBwdTile ? Nk - j * kBwdTile : kBwdTile;  // key rows of this tile
 
@@ -413,13 +419,16 @@ __global__ void __launch_bounds__(512, 1)
     uint8_t* ds_row = smem + L::kDSOff + h * L::kChunkBytes + r * 128;
     for (int it = 0; it < n_it; ++it) {
       const int i = i0 + it;
-      const bool diag = CAUSAL && i == j;
-      // Key row r sees query columns [lo, hi) of this tile: lo = r on the
-      // diagonal tile (key after query is masked), hi = the queries before
-      // Nq, and none at all if the key is past Nk.  P is zeroed outside.
+      // Key row r sees query q of this tile iff q >= dlt + r; the tile needs
+      // the causal test if its last key row does not see query 0.
+      const int dlt = (j - i) * kBwdTile - off;
+      const bool diag = CAUSAL && dlt + kBwdTile - 1 > 0;
+      // Key row r sees query columns [lo, hi) of this tile: lo from the
+      // causal mask, hi = the queries before Nq, and none at all if the key
+      // is past Nk.  P is zeroed outside.
       const int q_valid = Nq - i * kBwdTile;
       const bool masked = diag || kv_valid < kBwdTile || q_valid < kBwdTile;
-      const int lo = diag ? r : 0;
+      const int lo = diag && dlt + r > 0 ? dlt + r : 0;
       const int hi = r < kv_valid ? (q_valid < kBwdTile ? q_valid : kBwdTile) : 0;
       const uint32_t span = hi > lo ? static_cast<uint32_t>(hi - lo) : 0u;
       const int q_base = 64 * h - lo;  // column q tests (q - lo) < span, unsigned

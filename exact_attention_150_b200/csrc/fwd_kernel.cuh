@@ -79,7 +79,7 @@ template <int D, bool BF16, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o_ptr,
-               float* __restrict__ lse_ptr, int Nq, int Nk, float scale_log2) {
+               float* __restrict__ lse_ptr, int Nq, int Nk, int off, float scale_log2) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -108,8 +108,24 @@ __global__ void __launch_bounds__(384, 1)
   const int nkt = (Nk + kTile - 1) / kTile;
   // Causal: the heaviest query tiles are launched first.
   const int qt = CAUSAL ? (nqt - 1 - static_cast<int>(blockIdx.y)) : static_cast<int>(blockIdx.y);
-  // Key tiles this query tile sees (top-left causal: key <= query).
-  const int n = CAUSAL ? (qt + 1 < nkt ? qt + 1 : nkt) : nkt;
+  // Key tiles this query tile sees.  Causal: query i sees key k iff
+  // k <= i + off (off = 0 top-left, Nk - Nq bottom-right).
+  int n = nkt;
+  if (CAUSAL) {
+    const int last_row = qt * kTile + kTile - 1 < Nq - 1 ? qt * kTile + kTile - 1 : Nq - 1;
+    const int last_key = last_row + off < Nk - 1 ? last_row + off : Nk - 1;
+    n = last_key < 0 ? 0 : last_key / kTile + 1;
+  }
+  if (n == 0) {
+    // No row of this tile sees a key (bottom-right with Nq > Nk): the
+    // softmax is empty, O = 0 and LSE = log 0.
+    const int rows = Nq - qt * kTile < kTile ? Nq - qt * kTile : kTile;
+    const size_t grow0 = static_cast<size_t>(bh) * Nq + static_cast<size_t>(qt) * kTile;
+    for (int e = threadIdx.x; e < rows * D / 8; e += blockDim.x)
+      reinterpret_cast<uint4*>(o_ptr + grow0 * D)[e] = make_uint4(0u, 0u, 0u, 0u);
+    for (int e = threadIdx.x; e < rows; e += blockDim.x) lse_ptr[grow0 + e] = -INFINITY;
+    return;
+  }
 
   // Refuse to run (and report) if alignment left too little shared memory.
   if (static_cast<uint32_t>(smem - smem_raw) + L::kBytes > dynamic_smem_bytes()) {
@@ -323,12 +339,13 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 64; ++c) x[c] *= scale_log2;
       }
-      // Mask keys past Nk (ragged last tile) and, on the diagonal tile,
-      // keys after this query (the tiles start at the same offset).
+      // Mask keys past Nk (ragged last tile) and, causal, keys after
+      // query + off: column c is kept iff c <= lim.
       const int kv_valid = Nk - j * kTile;
-      if ((CAUSAL && j == qt) || kv_valid < kTile) {
+      const int diag_lim = (qt - j) * kTile + off;  // lim of row 0 from the mask
+      if ((CAUSAL && diag_lim < kTile - 1) || kv_valid < kTile) {
         int lim = kv_valid - 1;
-        if (CAUSAL && j == qt && row < lim) lim = row;
+        if (CAUSAL && diag_lim + row < lim) lim = diag_lim + row;
 #pragma unroll
         for (int c = 0; c < 64; ++c)
           if (64 * h + c > lim) x[c] = -INFINITY;
@@ -379,7 +396,10 @@ __global__ void __launch_bounds__(384, 1)
       float2 su[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) su[i] = make_float2(0.f, 0.f);
-      const float2 cx2 = make_float2(cx, cx), negm2 = make_float2(-m_run, -m_run);
+      // A row that has seen no key yet (m_run = -inf; causal with off < 0)
+      // uses 0: its scores are all -inf, so p = 0 rather than NaN.
+      const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      const float2 cx2 = make_float2(cx, cx), negm2 = make_float2(-m_use, -m_use);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
@@ -409,7 +429,13 @@ __global__ void __launch_bounds__(384, 1)
     if (ok && n > 0) {
       tc_fence_after();
       const float l_tot = l_run + xsum[(h ^ 1) * kTile + row];
-      const float inv = 1.f / __uint_as_float(tmem_ld1(t_row + L::kColL));
+      // A row that sees no key keeps m_run = -inf: O = 0 and LSE = -inf.
+      // (Its sums are not exactly 0: the FMA-pipe exponential returns
+      // ~2^-126 rather than 0 for a masked score.)
+      // (tcgen05.ld is warp-collective: every lane loads, then selects.)
+      const bool empty = m_run == -INFINITY;
+      const float l_tc = __uint_as_float(tmem_ld1(t_row + L::kColL));
+      const float inv = empty ? 0.f : 1.f / l_tc;
       const bool live = qt * kTile + row < Nq;  // padding rows of a ragged tile are not stored
       const size_t grow = static_cast<size_t>(bh) * Nq + static_cast<size_t>(qt) * kTile + row;
       uint4* dst = reinterpret_cast<uint4*>(o_ptr + grow * D + (D / 2) * h);
@@ -426,7 +452,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int v = 0; v < 4; ++v) dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
-      if (h == 0 && live) lse_ptr[grow] = (m_run + lg2(l_tot)) * 0.69314718055994530942f;
+      if (h == 0 && live) lse_ptr[grow] = empty ? -INFINITY : (m_run + lg2(l_tot)) * 0.69314718055994530942f;
     }
   }
 

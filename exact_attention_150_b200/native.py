@@ -22,6 +22,8 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "attn.h")
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_SCRATCH_LIMIT, ATTN_ERR_SMEM = range(7)
 ATTN_FP16, ATTN_BF16 = 0, 1
 ATTN_BWD_ALL, ATTN_BWD_PREPROCESS, ATTN_BWD_MAIN, ATTN_BWD_CONVERT = range(4)
+ATTN_CAUSAL_NONE, ATTN_CAUSAL_TOP_LEFT, ATTN_CAUSAL_BOTTOM_RIGHT = range(3)
+_CAUSAL_NAMES = {"none": ATTN_CAUSAL_NONE, "top_left": ATTN_CAUSAL_TOP_LEFT, "bottom_right": ATTN_CAUSAL_BOTTOM_RIGHT}
 
 _lib = None
 
@@ -139,7 +141,17 @@ def _check_tensor(name: str, t: torch.Tensor, shape, dtype) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
-def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None):
+def causal_code(causal) -> int:
+    """The C ABI's `causal` value: False/True (top-left), an attn_causal
+    integer, or "none" / "top_left" / "bottom_right"."""
+    if isinstance(causal, str):
+        if causal not in _CAUSAL_NAMES:
+            raise ValueError(f"causal must be one of {sorted(_CAUSAL_NAMES)}, got {causal!r}")
+        return _CAUSAL_NAMES[causal]
+    return int(causal)
+
+
+def forward(q, k, v, causal=False, scale: float | None = None, out=None, lse=None, stream=None):
     """O, LSE = attention(q, k, v) for q [B,H,Nq,d], k and v [B,H,Nk,d]."""
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
@@ -158,11 +170,11 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     _check("attn_fwd", attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                B, H, Nq, Nk, d, float(scale), causal, code, stream))
+                                B, H, Nq, Nk, d, float(scale), causal_code(causal), code, stream))
     return out, lse
 
 
-def backward(q, k, v, out, lse, dout, causal: bool = False, scale: float | None = None,
+def backward(q, k, v, out, lse, dout, causal=False, scale: float | None = None,
              dq=None, dk=None, dv=None, workspace=None, stream=None, phase: int = ATTN_BWD_ALL):
     """dQ, dK, dV of attention for the output gradient dout.  `phase` runs
     only one of the three backward kernels (see attn_bwd_phase)."""
@@ -189,7 +201,7 @@ def backward(q, k, v, out, lse, dout, causal: bool = False, scale: float | None 
         stream = torch.cuda.current_stream(q.device).cuda_stream
     _check("attn_bwd", attn_bwd_phase(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                       dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                                      workspace.data_ptr(), B, H, Nq, Nk, d, float(scale), causal, code, phase,
+                                      workspace.data_ptr(), B, H, Nq, Nk, d, float(scale), causal_code(causal), code, phase,
                                       stream))
     return dq, dk, dv
 

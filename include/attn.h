@@ -24,11 +24,15 @@
  *   allocation of its own between calls.
  * Stream.  `stream` is a cudaStream_t (NULL = legacy default stream).  Every
  *   call only enqueues work on it and returns without synchronising.
- * Mask.  causal != 0 applies the top-left causal mask: query row i attends to
- *   key row j iff j <= i.  (The pages name a causal mask but not its
- *   alignment when Nq != Nk; top-left is the reading taken.  With Nq > Nk the
- *   query rows past Nk see every key; with Nq < Nk the keys past Nq are seen
- *   by no query, and their dK, dV are zero.)
+ * Mask.  `causal` is an attn_causal value; anything else returns
+ *   ATTN_ERR_INVALID_ARG.  ATTN_CAUSAL_TOP_LEFT (1): query row i attends to
+ *   key row j iff j <= i.  ATTN_CAUSAL_BOTTOM_RIGHT (2): iff j <= i + Nk - Nq,
+ *   so the last query row sees every key (a block of new queries appended
+ *   after Nk - Nq cached keys).  The two agree when Nq == Nk.  (The pages name
+ *   a causal mask but not its alignment when Nq != Nk; top-left is the
+ *   default reading, bottom-right the option.)  Keys that no query sees get
+ *   dK = dV = 0.  A query row that sees no key (bottom-right with Nq > Nk:
+ *   rows i < Nq - Nk) has an empty softmax: O = 0, LSE = -inf, dQ = 0.
  * LSE.  lse[b][h][i] = ln sum_j exp(scale * q_i . k_j) over the unmasked j:
  *   the natural-log row log-sum-exp of the scaled scores, in fp32.
  * Supported shapes.  d in {64, 128}; any Nq, Nk >= 0 (the kernels work in
@@ -73,6 +77,13 @@ typedef enum {
 } attn_status;
 
 typedef enum { ATTN_FP16 = 0, ATTN_BF16 = 1 } attn_dtype;
+
+/* Values of the `causal` argument (see Mask above). */
+typedef enum {
+  ATTN_CAUSAL_NONE = 0,
+  ATTN_CAUSAL_TOP_LEFT = 1,
+  ATTN_CAUSAL_BOTTOM_RIGHT = 2
+} attn_causal;
 
 /*
  * Forward pass.  Writes O = softmax(scale * Q K^T [+ causal mask]) V (16-bit,

@@ -52,7 +52,11 @@ def assert_o(got, ref, dtype, what=""):
 
 
 def assert_lse(got, ref, what=""):
-    err = float(np.max(np.abs(got - ref), initial=0.0))
+    # Rows that see no key have LSE = -inf on both sides; compare the rest.
+    inf_got, inf_ref = np.isinf(got), np.isinf(ref)
+    assert np.array_equal(inf_got, inf_ref) and np.array_equal(got[inf_ref], ref[inf_ref]), \
+        f"{what}: infinite LSE entries differ"
+    err = float(np.max(np.abs(got[~inf_ref] - ref[~inf_ref]), initial=0.0))
     assert err <= LSE_TOL, f"{what}: LSE max abs err {err:.3e}"
 
 
@@ -61,22 +65,33 @@ def assert_grad(got, ref, name, what=""):
     assert e <= GRAD_TOL, f"{what}: {name} relative Frobenius error {e:.3e}"
 
 
+def oracle_mask(causal, nq: int, nk: int) -> tuple[bool, int]:
+    """The oracle's (causal, q_offset) for the library's `causal` argument:
+    top-left is offset 0, bottom-right is offset Nk - Nq."""
+    if causal in ("bottom_right", 2):
+        return True, nk - nq
+    if causal in ("none", False, 0):
+        return False, 0
+    return True, 0
+
+
 def oracle_forward_slices(q, k, v, scale, causal, slices, rows=None):
     """Oracle O and LSE for the given flat (b*h) slices, optionally only for
     query rows `rows` (absolute indices, ascending)."""
     B, H, Nq, d = q.shape
+    causal, off = oracle_mask(causal, Nq, k.shape[2])
     qf, kf, vf = (t.reshape(B * H, t.shape[2], d) for t in (q, k, v))
     outs, lses = [], []
     for s in slices:
         k64, v64 = f64(kf[s]), f64(vf[s])
         if rows is None:
-            o, lse, _ = oracle.forward(f64(qf[s]), k64, v64, scale, causal)
+            o, lse, _ = oracle.forward(f64(qf[s]), k64, v64, scale, causal, q_offset=off)
         else:
             o = np.empty((len(rows), d))
             lse = np.empty(len(rows))
             q64 = f64(qf[s])
             for r in rows:  # one row at a time: the oracle sees exactly that query
-                oo, ll, _ = oracle.forward(q64[r:r + 1], k64, v64, scale, causal, q_offset=r)
+                oo, ll, _ = oracle.forward(q64[r:r + 1], k64, v64, scale, causal, q_offset=r + off)
                 i = rows.index(r)
                 o[i], lse[i] = oo[0], ll[0]
         outs.append(o)

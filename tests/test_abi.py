@@ -149,3 +149,21 @@ def test_bwd_phase_validates_like_bwd(lib):
     assert native.attn_bwd_phase(**args) == native.ATTN_ERR_INVALID_ARG
     args.update(B=0)
     assert native.attn_bwd_phase(**args) == native.ATTN_OK
+
+
+@pytest.mark.parametrize("causal", [-1, 3, 99])
+def test_causal_value_out_of_range(lib, causal):
+    assert _fwd(causal=causal) == native.ATTN_ERR_INVALID_ARG
+    assert _bwd(causal=causal) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd(causal=causal, B=0) == native.ATTN_ERR_INVALID_ARG  # validated before the empty-problem exit
+
+
+def test_causal_codes_match_the_header():
+    import re
+    text = open(native.HEADER).read()
+    values = {m.group(1): int(m.group(2)) for m in re.finditer(r"(ATTN_CAUSAL_\w+)\s*=\s*(\d+)", text)}
+    assert values == {"ATTN_CAUSAL_NONE": native.ATTN_CAUSAL_NONE, "ATTN_CAUSAL_TOP_LEFT": native.ATTN_CAUSAL_TOP_LEFT,
+                      "ATTN_CAUSAL_BOTTOM_RIGHT": native.ATTN_CAUSAL_BOTTOM_RIGHT}
+    assert [native.causal_code(c) for c in (False, True, "none", "top_left", "bottom_right", 2)] == [0, 1, 0, 1, 2, 2]
+    with pytest.raises(ValueError):
+        native.causal_code("bottom-left")

@@ -40,8 +40,9 @@ def check_grads_all_slices(q, k, v, do, causal, scale, what):
     flat = lambda t, n: t.reshape(B * H, n, d)
     for s in range(B * H):
         args = [parity.f64(flat(t, n)[s]) for t, n in ((q, Nq), (k, Nk), (v, Nk), (do, Nq))]
-        ro, rlse, _ = oracle.forward(*args[:3], scale, causal)
-        rdq, rdk, rdv = oracle.backward(*args, scale, causal)
+        oc, off = parity.oracle_mask(causal, Nq, Nk)
+        ro, rlse, _ = oracle.forward(*args[:3], scale, oc, off)
+        rdq, rdk, rdv = oracle.backward(*args, scale, oc, off)
         tag = f"{what} slice {s}"
         parity.assert_o(parity.f64(flat(o, Nq)[s]), ro, q.dtype, tag)
         parity.assert_lse(parity.f64(lse.reshape(B * H, Nq)[s]), rlse, tag)
@@ -80,6 +81,20 @@ def test_backward_ragged_nq_ne_nk(causal, nq, nk):
     """Includes key tiles no query sees (causal, Nk > Nq): their dK, dV are 0."""
     q, k, v, do = draw(1, 2, nq, nk, 64, torch.float16, seed=31 + nq + nk, with_grad=True)
     check_grads_all_slices(q, k, v, do, causal, 0.125, f"Nq{nq} Nk{nk} causal={causal}")
+
+
+@pytest.mark.parametrize("nq,nk", [(100, 300), (300, 100), (1, 257), (257, 1), (128, 384), (384, 128),
+                                   (200, 640), (129, 129)])
+def test_backward_bottom_right(nq, nk):
+    """Bottom-right causal: query i sees keys j <= i + Nk - Nq.  With Nq > Nk
+    the first Nq - Nk query rows see no key: their dQ is 0."""
+    q, k, v, do = draw(1, 2, nq, nk, 128, torch.bfloat16, seed=41 + nq + nk, with_grad=True)
+    check_grads_all_slices(q, k, v, do, "bottom_right", 1 / math.sqrt(128), f"bottom-right Nq{nq} Nk{nk}")
+
+
+def test_backward_bottom_right_d64_fp16():
+    q, k, v, do = draw(2, 2, 300, 700, 64, torch.float16, seed=43, with_grad=True)
+    check_grads_all_slices(q, k, v, do, "bottom_right", 0.125, "bottom-right d64 fp16")
 
 
 def test_backward_no_queries_gives_zero_dk_dv():

@@ -112,6 +112,35 @@ def test_forward_ragged_nq_ne_nk(causal, nq, nk):
     check_all_slices(q, k, v, causal, 1.0 / math.sqrt(128), f"Nq{nq} Nk{nk} causal={causal}")
 
 
+@pytest.mark.parametrize("nq,nk", [(100, 300), (300, 100), (1, 257), (257, 1), (128, 384), (384, 128),
+                                   (640, 200), (200, 640), (129, 129)])
+def test_forward_bottom_right(nq, nk):
+    """Bottom-right causal: query i sees keys j <= i + Nk - Nq.  With Nq > Nk
+    the first Nq - Nk rows see no key: O = 0 and LSE = -inf (whole query
+    tiles of such rows are written without any MMA)."""
+    q, k, v = draw(2, 2, nq, nk, 128, torch.bfloat16, seed=23 + nq + nk)
+    check_all_slices(q, k, v, "bottom_right", 1.0 / math.sqrt(128), f"bottom-right Nq{nq} Nk{nk}")
+    if nq > nk:
+        o, lse = run_forward(q, k, v, "bottom_right", 0.1)
+        assert torch.count_nonzero(o[:, :, :nq - nk]) == 0
+        assert torch.all(lse[:, :, :nq - nk] == float("-inf"))
+        assert torch.all(torch.isfinite(lse[:, :, nq - nk:]))
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.float16, 64), (torch.bfloat16, 64), (torch.float16, 128)])
+def test_forward_bottom_right_dtypes(dtype, d):
+    q, k, v = draw(1, 3, 333, 1000, d, dtype, seed=29)
+    check_all_slices(q, k, v, "bottom_right", 1.0 / math.sqrt(d), f"bottom-right d{d} {dtype}")
+
+
+def test_forward_bottom_right_single_query_is_noncausal():
+    """One new query after Nk - 1 cached keys sees all of them."""
+    q, k, v = draw(1, 4, 1, 1000, 128, torch.bfloat16, seed=31)
+    a = run_forward(q, k, v, "bottom_right", 0.088)
+    b = run_forward(q, k, v, False, 0.088)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
 def test_forward_empty_problems():
     for shape_q, shape_k in (((0, 2, 128, 64), (0, 2, 128, 64)), ((1, 2, 0, 64), (1, 2, 64, 64))):
         q = torch.zeros(shape_q, dtype=torch.bfloat16, device=DEV)
