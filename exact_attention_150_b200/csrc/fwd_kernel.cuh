@@ -10,9 +10,10 @@
 // page "Flash Attention 落地评估" (section 4); S never leaves the SM.
 //
 // Both products read their A operand from tensor memory (Q for S = Q K^T,
-// P for O += P V) and stream only K or V from shared memory: an MMA whose
-// two operands both come from shared memory runs at about half rate on
-// B200, one with A in tensor memory at full rate.
+// P for O += P V) and stream only K or V from shared memory.  A 128x128x16
+// MMA with both operands in shared memory reads 8 KB in its 64 cycles, all
+// of the SM's shared-memory bandwidth; with A in tensor memory it needs half,
+// which leaves room for the TMA writes of the K/V ring.
 //
 // CTA layout (384 threads, one CTA per SM):
 //   warp 0       TMA producer: Q once, then K_0, K_1, V_0, K_2, V_1, ...
