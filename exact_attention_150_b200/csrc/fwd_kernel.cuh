@@ -357,12 +357,41 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int c = 8; c < 64; c += 2) mp[(c >> 1) & 7] = max3f(mp[(c >> 1) & 7], x[c], x[c + 1]);
       float mx = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+      // Exponentials, sums and the in-place 16-bit P of this warpgroup's 64
+      // columns against the maximum m_run.  l_run sums the fp32
+      // probabilities (for LSE); the tensor core sums the rounded 16-bit ones
+      // (L).  Arguments and sums as packed fp32x2; one pair in four goes to
+      // the FMA-pipe exponential, since MUFU throughput bounds them otherwise.
+      // A row that has seen no key yet (m_run = -inf; causal with off < 0)
+      // uses 0: its scores are all -inf, so p = 0 rather than NaN.
+      float2 su[4];
+#define ATTN_EXP_STORE()                                                                            \
+  {                                                                                                 \
+    _Pragma("unroll") for (int i = 0; i < 4; ++i) su[i] = make_float2(0.f, 0.f);                    \
+    const float m_use = m_run == -INFINITY ? 0.f : m_run;                                           \
+    const float2 cx2 = make_float2(cx, cx), negm2 = make_float2(-m_use, -m_use);                    \
+    _Pragma("unroll") for (int c = 0; c < 2; ++c) {                                                 \
+      uint32_t pk[16];                                                                              \
+      _Pragma("unroll") for (int i = 0; i < 16; ++i) {                                              \
+        const float2 a = fma2(make_float2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), cx2, negm2);   \
+        const float2 p = ((i & 3) == 3) ? exp2_poly2(a) : make_float2(ex2(a.x), ex2(a.y));          \
+        pk[i] = pack2<BF16>(p.x, p.y);                                                              \
+        su[i & 3] = add2(su[i & 3], p);                                                             \
+      }                                                                                             \
+      tmem_st16(s_col + 16 * c, pk);                                                                \
+    }                                                                                               \
+  }
       // Row maximum over both halves of the key tile, exchanged through
       // shared memory (double-buffered by tile parity: a warpgroup cannot
       // rewrite a slot before the other has passed the next exchange, which
       // it reaches only after reading the slot).
       xchg[(b * 2 + h) * kTile + row] = mx;
       mbar_arrive(&xmax_bar[b]);
+      // After the first tile, compute P against the current maximum while
+      // the other warpgroup's half arrives: it stands unless the maximum has
+      // grown by more than 2^8 (then it is recomputed below; P is not read
+      // before p_full).
+      if (j > 0) ATTN_EXP_STORE()
       ok = __all_sync(0xffffffffu, mbar_wait(&xmax_bar[b], (j >> 1) & 1, abort_flag));
       if (!ok) break;
       mx = fmaxf(mx, xchg[(b * 2 + (h ^ 1)) * kTile + row]);
@@ -372,7 +401,8 @@ __global__ void __launch_bounds__(384, 1)
       // warpgroups see the same m_run and m_new, so they decide alike.
       const bool need = (j > 0) && (m_new - m_run > 8.f);
       if (j == 0) m_run = m_new;
-      if (__any_sync(0xffffffffu, need)) {
+      const bool any_need = __any_sync(0xffffffffu, need);
+      if (any_need) {
         // O must hold PV(j-1) complete before it is rescaled.
         ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, abort_flag));
         if (!ok) break;
@@ -392,29 +422,13 @@ __global__ void __launch_bounds__(384, 1)
           m_run = m_new;
         }
       }
-      // l_run sums the fp32 probabilities (for LSE); the tensor core sums
-      // the rounded 16-bit ones (L).  Arguments and sums as packed fp32x2.
-      float2 su[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) su[i] = make_float2(0.f, 0.f);
-      // A row that has seen no key yet (m_run = -inf; causal with off < 0)
-      // uses 0: its scores are all -inf, so p = 0 rather than NaN.
-      const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      const float2 cx2 = make_float2(cx, cx), negm2 = make_float2(-m_use, -m_use);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float2 a = fma2(make_float2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), cx2, negm2);
-          // One pair in four on the FMA pipe: MUFU throughput bounds the
-          // exponentials otherwise.
-          const float2 p = ((i & 3) == 3) ? exp2_poly2(a) : make_float2(ex2(a.x), ex2(a.y));
-          pk[i] = pack2<BF16>(p.x, p.y);
-          su[i & 3] = add2(su[i & 3], p);
-        }
-        tmem_st16(s_col + 16 * c, pk);
+      // First tile, or a maximum that moved: (re)compute against the final
+      // m_run (rows of the warp whose m_run did not move get the same values).
+      if (j == 0 || any_need) {
+        if (j > 0) tmem_st_wait();  // the optimistic stores land before they are overwritten
+        ATTN_EXP_STORE()
       }
+#undef ATTN_EXP_STORE
       const float2 su01 = add2(su[0], su[1]), su23 = add2(su[2], su[3]);
       l_run += (su01.x + su01.y) + (su23.x + su23.y);
       tmem_st_wait();
