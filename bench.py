@@ -56,6 +56,8 @@ def parse_args(argv=None):
     p.add_argument("--seq", type=int, default=None, help="override the sequence length (profiling runs)")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--deterministic", action="store_true",
+                   help="time the bit-reproducible backward (attn_bwd_deterministic) instead of attn_bwd")
     return p.parse_args(argv)
 
 
@@ -257,7 +259,7 @@ def run_ours(args):
 
     def bwd(phase):
         native.backward(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, dq=dq, dk=dk, dv=dv, workspace=ws,
-                        phase=phase)
+                        phase=phase, deterministic=args.deterministic and phase == native.ATTN_BWD_ALL)
 
     def step(ev=None):
         if ev is not None:
@@ -269,6 +271,13 @@ def run_ours(args):
             return
         if ev is not None:
             ev[1].record(stream)
+        if args.deterministic:
+            # One call: order counters, preprocess, main and convert kernels.
+            bwd(native.ATTN_BWD_ALL)
+            if ev is not None:
+                for e in ev[2:]:
+                    e.record(stream)
+            return
         bwd(native.ATTN_BWD_PREPROCESS)
         if ev is not None:
             ev[2].record(stream)
@@ -279,7 +288,7 @@ def run_ours(args):
         if ev is not None:
             ev[4].record(stream)
 
-    launches_per_step = 4 if w.backward else 1
+    launches_per_step = (5 if args.deterministic else 4) if w.backward else 1
     for _ in range(max(args.warmup, 0)):
         step()
     torch.cuda.synchronize(device)
@@ -308,7 +317,12 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     kernels = {"fwd_kernel": {"ms": fwd_ms, "tflops": w.fwd_flops() / fwd_ms / 1e9}}
-    if w.backward:
+    if w.backward and args.deterministic:
+        det_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        kernels["bwd_deterministic (order counters + 3 kernels)"] = {"ms": det_ms,
+                                                                      "tflops": w.bwd_flops() / det_ms / 1e9}
+        dom_name, dom_ms, dom_flops = "bwd_deterministic", det_ms, w.bwd_flops()
+    elif w.backward:
         pre_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
         main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
         post_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
@@ -325,7 +339,7 @@ def run_ours(args):
     achieved = dom_flops / dom_ms / 1e9
     traffic = None
     if BWD_MAIN_TRAFFIC is not None and dom_name == "bwd_main_kernel":
-        traffic = BWD_MAIN_TRAFFIC.get((w.N, w.H))
+        traffic = BWD_MAIN_TRAFFIC.get((w.N, w.H)) if not args.deterministic else None
 
     # End to end through the public API: pinned host inputs -> device, the
     # forward and backward calls, results -> pinned host, every step.
@@ -342,7 +356,7 @@ def run_ours(args):
                 dst.copy_(src, non_blocking=True)
             fwd()
             if w.backward:
-                bwd(native.ATTN_BWD_ALL)
+                bwd(native.ATTN_BWD_ALL)  # deterministic when --deterministic
             for dst, src in zip(outs_h, (o, lse, dq, dk, dv)):
                 dst.copy_(src, non_blocking=True)
 
@@ -377,7 +391,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp16",
         "data": "synthetic: seeded i.i.d. N(0,1) Q, K, V, dO (x%g)" % w.input_scale,
-        "config": config_of(w, world),
+        "config": {**config_of(w, world), **({"backward": "deterministic"} if args.deterministic else {})},
         "fwd_tflops": w.fwd_flops() / fwd_ms / 1e9,
         "bwd_tflops": (w.bwd_flops() / (max_ms / args.steps - fwd_ms) / 1e9) if w.backward else None,
         "kernels": kernels,

@@ -60,6 +60,15 @@ int tiles(int n) { return (n + kTile - 1) / kTile; }
 // the last slice they land here.
 long long pad_rows(int Nq) { return static_cast<long long>(tiles(Nq)) * kTile - Nq; }
 
+// Workspace layout: dQ accumulator [(B*H*Nq + pad_rows) * d] | D [B*H*Nq] |
+// -log2(e) LSE [B*H*Nq] | (16-byte aligned) order counters [B*H][tiles(Nq)]
+// of the deterministic backward.
+long long counters_offset_floats(int BH, int Nq, int d) {
+  const long long rows = static_cast<long long>(BH) * Nq;
+  const long long f = (rows + pad_rows(Nq)) * d + 2 * rows;
+  return (f + 3) / 4 * 4;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Sizes may be zero (an empty problem); they may not be negative.
@@ -92,7 +101,7 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool DET>
 attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                        const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv, float* ws,
                        int BH, int Nq, int Nk, int off, float scale, int phase, cudaStream_t st) {
@@ -101,8 +110,11 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   float* dqacc = ws;
   float* dvec = ws + (qrows + pad_rows(Nq)) * D;
   float* nlse2 = dvec + qrows;
+  int* dq_order = DET ? reinterpret_cast<int*>(ws + counters_offset_floats(BH, Nq, D)) : nullptr;
 
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_PREPROCESS) {
+    if (DET && cudaMemsetAsync(dq_order, 0, static_cast<size_t>(BH) * tiles(Nq) * sizeof(int), st) != cudaSuccess)
+      return ATTN_ERR_CUDA;
     constexpr int kRowsPerBlock = 256 / (D / 8);
     const long long pre_blocks = (qrows + kRowsPerBlock - 1) / kRowsPerBlock;
     attn::bwd_pre_kernel<D, BF16><<<static_cast<unsigned>(pre_blocks), 256, 0, st>>>(
@@ -110,11 +122,12 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_MAIN) {
-    auto kern = attn::bwd_main_kernel<D, BF16, CAUSAL>;
+    auto kern = attn::bwd_main_kernel<D, BF16, CAUSAL, DET>;
     if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
     dim3 grid(BH, tiles(Nk));
     kern<<<grid, 512, L::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, dqacc, static_cast<uint16_t*>(dk),
-                                       static_cast<uint16_t*>(dv), Nq, Nk, off, scale, scale * 1.4426950408889634f);
+                                       static_cast<uint16_t*>(dv), dq_order, Nq, Nk, off, scale,
+                                       scale * 1.4426950408889634f);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_CONVERT) {
@@ -140,16 +153,23 @@ attn_status dispatch_fwd_causal(int causal, const CUtensorMap& mq, const CUtenso
 }
 
 template <int D, bool BF16>
-attn_status dispatch_bwd_causal(int causal, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                                const CUtensorMap& mdo, const void* o, const void* dout, const float* lse, void* dq,
-                                void* dk, void* dv, float* ws, int BH, int Nq, int Nk, float scale, int phase,
-                                cudaStream_t st) {
+attn_status dispatch_bwd_causal(int causal, bool det, const CUtensorMap& mq, const CUtensorMap& mk,
+                                const CUtensorMap& mv, const CUtensorMap& mdo, const void* o, const void* dout,
+                                const float* lse, void* dq, void* dk, void* dv, float* ws, int BH, int Nq, int Nk,
+                                float scale, int phase, cudaStream_t st) {
   const int off = causal_offset(causal, Nq, Nk);
-  return causal
-             ? launch_bwd<D, BF16, true>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, off, scale, phase, st)
-             : launch_bwd<D, BF16, false>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, off, scale, phase,
-                                          st);
+#define ATTN_LAUNCH_BWD(C, DT) \
+  launch_bwd<D, BF16, C, DT>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, off, scale, phase, st)
+  if (det) return causal ? ATTN_LAUNCH_BWD(true, true) : ATTN_LAUNCH_BWD(false, true);
+  return causal ? ATTN_LAUNCH_BWD(true, false) : ATTN_LAUNCH_BWD(false, false);
+#undef ATTN_LAUNCH_BWD
 }
+
+// The backward phases shared by attn_bwd_phase (det = false) and
+// attn_bwd_deterministic (det = true).
+attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
+                     int causal, attn_dtype dtype, int phase, bool det, void* stream);
 
 }  // namespace
 
@@ -216,11 +236,11 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
 
 size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
   if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return 0;  // empty problems need none
-  const unsigned long long rows = static_cast<unsigned long long>(B) * H * Nq;
-  const unsigned long long floats =
-      (rows + static_cast<unsigned long long>(pad_rows(Nq))) * static_cast<unsigned long long>(d) + 2 * rows;
-  if (floats > (~0ull) / 4) return 0;
-  return static_cast<size_t>(floats * 4);
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh > 0x7fffffffLL || bh * Nq > (1LL << 40)) return 0;
+  const unsigned long long words = static_cast<unsigned long long>(counters_offset_floats(static_cast<int>(bh), Nq, d)) +
+                                   static_cast<unsigned long long>(bh) * tiles(Nq);
+  return static_cast<size_t>(words * 4);
 }
 
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
@@ -233,6 +253,24 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
 attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const void* o, const float* lse,
                            const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq,
                            int Nk, int d, float scale, int causal, attn_dtype dtype, int phase, void* stream) {
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, causal, dtype, phase, false,
+                  stream);
+}
+
+attn_status attn_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                   const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H,
+                                   int Nq, int Nk, int d, float scale, int causal, attn_dtype dtype, void* stream) {
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, causal, dtype, ATTN_BWD_ALL,
+                  true, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
+                     int causal, attn_dtype dtype, int phase, bool det, void* stream) {
   if (phase < ATTN_BWD_ALL || phase > ATTN_BWD_CONVERT) return ATTN_ERR_INVALID_ARG;
   const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
@@ -260,12 +298,16 @@ attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const vo
     return ATTN_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
-  if (d == 64)
-    return bf16 ? dispatch_bwd_causal<64, true>(causal, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st)
-                : dispatch_bwd_causal<64, false>(causal, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st);
-  return bf16 ? dispatch_bwd_causal<128, true>(causal, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st)
-              : dispatch_bwd_causal<128, false>(causal, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st);
+#define ATTN_DISPATCH_BWD(DD, BB) \
+  dispatch_bwd_causal<DD, BB>(causal, det, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st)
+  if (d == 64) return bf16 ? ATTN_DISPATCH_BWD(64, true) : ATTN_DISPATCH_BWD(64, false);
+  return bf16 ? ATTN_DISPATCH_BWD(128, true) : ATTN_DISPATCH_BWD(128, false);
+#undef ATTN_DISPATCH_BWD
 }
+
+}  // namespace
+
+extern "C" {
 
 attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                              const void* dout, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d,

@@ -136,13 +136,38 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-template <int D, bool BF16, bool CAUSAL>
+// Deterministic dQ: waits until *turn >= target (acquire), with the same
+// time limit and abort protocol as the mbarrier waits.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool wait_turn(const int* turn, int target, volatile int* abort) {
+  if (ld_acquire_gpu(turn) >= target) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+      __nanosleep(64);
+      if (ld_acquire_gpu(turn) >= target) return true;
+    }
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      atomicExch(&g_device_status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+template <int D, bool BF16, bool CAUSAL, bool DET>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const float* __restrict__ dvec, const float* __restrict__ nlse2, float* __restrict__ dqacc,
-                    uint16_t* __restrict__ dk_ptr, uint16_t* __restrict__ dv_ptr, int Nq, int Nk, int off,
-                    float scale, float scale_log2) {
+                    uint16_t* __restrict__ dk_ptr, uint16_t* __restrict__ dv_ptr, int* __restrict__ dq_order,
+                    int Nq, int Nk, int off, float scale, float scale_log2) {
   using L = BwdLayout<D>;
   constexpr bool kDqT = (D == 128);  // dQ formed transposed (see above)
   constexpr uint32_t kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 256 + D;
@@ -510,6 +535,29 @@ __global__ void __launch_bounds__(512, 1)
       if (!ok) break;
       tc_fence_after();
       const size_t qrow0 = static_cast<size_t>(bh) * Nq + static_cast<size_t>(i0 + it) * kBwdTile;
+      // Deterministic mode: the key tiles that reach a query tile are a
+      // prefix 0..J of the key tiles (the first query tile a key tile sees
+      // never decreases with it), so this CTA is contributor number j of
+      // every query tile it covers.  It reduces into the tile only after the
+      // 4 drain warps of contributors 0..j-1 have each counted theirs.
+      int* turn = DET ? dq_order + static_cast<size_t>(bh) * nqt + (i0 + it) : nullptr;
+      auto await_turn = [&]() {
+        if constexpr (DET) {
+          if (!__all_sync(0xffffffffu, wait_turn(turn, 4 * j, abort_flag))) return false;
+          __threadfence();
+        }
+        return true;
+      };
+      auto pass_turn = [&]() {
+        if constexpr (DET) {
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence();
+            atomicAdd(turn, 1);
+          }
+        }
+      };
       if constexpr (kDqT) {
         // Thread = head-dim index d; a warp's reduction covers 32 consecutive
         // d of one query row (128 contiguous bytes).
@@ -525,6 +573,8 @@ __global__ void __launch_bounds__(512, 1)
         tmem_ld32(t_row + kColDQ + 96, vd);
         tc_fence_before();
         mbar_arrive(dq_free);
+        ok = await_turn();
+        if (!ok) break;
 #pragma unroll
         for (int q = 0; q < 32; ++q)
           atomicAdd(base + static_cast<size_t>(q) * D, __uint_as_float(va[q]) * scale);
@@ -537,6 +587,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int q = 0; q < 32; ++q)
           atomicAdd(base + static_cast<size_t>(96 + q) * D, __uint_as_float(vd[q]) * scale);
+        pass_turn();
       } else {
         // Thread = query row; 64 head-dim values as 16-byte vector reductions.
         uint32_t va[32], vb[32];
@@ -544,6 +595,8 @@ __global__ void __launch_bounds__(512, 1)
         tmem_ld32(t_row + kColDQ + 32, vb);
         tc_fence_before();
         mbar_arrive(dq_free);
+        ok = await_turn();
+        if (!ok) break;
         float* dst = dqacc + (qrow0 + row) * D;
 #pragma unroll
         for (int v = 0; v < 8; ++v)
@@ -555,6 +608,7 @@ __global__ void __launch_bounds__(512, 1)
           atomicAdd(reinterpret_cast<float4*>(dst + 32 + 4 * v),
                     make_float4(__uint_as_float(vb[4 * v]) * scale, __uint_as_float(vb[4 * v + 1]) * scale,
                                 __uint_as_float(vb[4 * v + 2]) * scale, __uint_as_float(vb[4 * v + 3]) * scale));
+        pass_turn();
       }
     }
     if (ok && n_it > 0) {

@@ -51,6 +51,8 @@ def load() -> ctypes.CDLL:
     lib.attn_bwd.restype = st
     lib.attn_bwd_phase.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
     lib.attn_bwd_phase.restype = st
+    lib.attn_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+    lib.attn_bwd_deterministic.restype = st
     lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
     lib.attn_bwd_noalloc.restype = st
     lib.attn_bwd_noalloc_max_scratch_bytes.argtypes = []
@@ -96,6 +98,13 @@ def attn_bwd_phase(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d
     """Direct call of attn_bwd_phase (one of the three backward kernels)."""
     return load().attn_bwd_phase(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale,
                                  int(causal), dtype, phase, stream)
+
+
+def attn_bwd_deterministic(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, causal, dtype,
+                           stream) -> int:
+    """Direct call of attn_bwd_deterministic (bit-reproducible dQ)."""
+    return load().attn_bwd_deterministic(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale,
+                                         int(causal), dtype, stream)
 
 
 def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
@@ -175,9 +184,11 @@ def forward(q, k, v, causal=False, scale: float | None = None, out=None, lse=Non
 
 
 def backward(q, k, v, out, lse, dout, causal=False, scale: float | None = None,
-             dq=None, dk=None, dv=None, workspace=None, stream=None, phase: int = ATTN_BWD_ALL):
+             dq=None, dk=None, dv=None, workspace=None, stream=None, phase: int = ATTN_BWD_ALL,
+             deterministic: bool = False):
     """dQ, dK, dV of attention for the output gradient dout.  `phase` runs
-    only one of the three backward kernels (see attn_bwd_phase)."""
+    only one of the three backward kernels (see attn_bwd_phase);
+    `deterministic` selects attn_bwd_deterministic (all phases)."""
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
     code = _dtype_code(q)
@@ -199,10 +210,16 @@ def backward(q, k, v, out, lse, dout, causal=False, scale: float | None = None,
         raise ValueError(f"workspace must be a CUDA buffer of at least {nbytes} bytes")
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
-    _check("attn_bwd", attn_bwd_phase(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                                      workspace.data_ptr(), B, H, Nq, Nk, d, float(scale), causal_code(causal), code, phase,
-                                      stream))
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr(), workspace.data_ptr())
+    if deterministic:
+        if phase != ATTN_BWD_ALL:
+            raise ValueError("the deterministic backward runs all phases")
+        _check("attn_bwd_deterministic",
+               attn_bwd_deterministic(*ptrs, B, H, Nq, Nk, d, float(scale), causal_code(causal), code, stream))
+    else:
+        _check("attn_bwd", attn_bwd_phase(*ptrs, B, H, Nq, Nk, d, float(scale), causal_code(causal), code, phase,
+                                          stream))
     return dq, dk, dv
 
 

@@ -103,12 +103,14 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
                      attn_dtype dtype, void* stream);
 
 /*
- * Size in bytes of the device workspace attn_bwd needs: an fp32 dQ
- * accumulator [B][H][Nq][d] followed by (128 - Nq % 128) % 128 rows of d
- * floats of padding (a ragged last query tile reduces its masked rows, which
- * are exact zeros, into them), then the fp32 row term D [B][H][Nq], then the
- * fp32 row term -log2(e) * LSE [B][H][Nq].  Returns 0 for an empty problem
- * (any size 0), a negative size, or a total that overflows size_t.
+ * Size in bytes of the device workspace attn_bwd and attn_bwd_deterministic
+ * need: an fp32 dQ accumulator [B][H][Nq][d] followed by
+ * (128 - Nq % 128) % 128 rows of d floats of padding (a ragged last query
+ * tile reduces its masked rows, which are exact zeros, into them), then the
+ * fp32 row term D [B][H][Nq], then the fp32 row term -log2(e) * LSE
+ * [B][H][Nq], then (16-byte aligned) B*H*ceil(Nq/128) int32 counters that
+ * order the deterministic backward's dQ reductions.  Returns 0 for an empty
+ * problem (any size 0), a negative size, or a total that overflows size_t.
  */
 size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d);
 
@@ -129,6 +131,23 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
                      void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
                      int causal, attn_dtype dtype, void* stream);
+
+/*
+ * attn_bwd with a bit-reproducible dQ.  The paper's backward has no such
+ * variant; the page "Flash Attention 落地评估" (section 4) raises
+ * reproducibility as a concern, and attn_bwd's dQ depends on the order in
+ * which fp32 atomic additions from different key tiles land.  Here the key
+ * tiles that reach a query tile add their dQ contributions in ascending
+ * key-tile order (each waits, with the same bounded wait as every other wait
+ * in these kernels, for a per-query-tile counter in the workspace), so two
+ * calls with the same inputs give identical dQ, dK and dV bits.  It is slower
+ * than attn_bwd: a key tile's reductions wait for the previous key tile's.
+ * Arguments, workspace and errors as for attn_bwd.
+ */
+attn_status attn_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                                   const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                   void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
+                                   int causal, attn_dtype dtype, void* stream);
 
 /*
  * One phase of attn_bwd, for callers that time or schedule the three

@@ -21,7 +21,7 @@ def lib():
 def test_header_declares_the_boundary():
     names = set(native.declared_symbols())
     assert {"attn_fwd", "attn_bwd", "attn_bwd_phase", "attn_bwd_workspace_bytes", "attn_last_device_status",
-            "attn_status_string"} <= names
+            "attn_status_string", "attn_bwd_deterministic"} <= names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -106,14 +106,35 @@ def test_unsupported_shapes(lib, kw):
     assert _bwd(**kw) == native.ATTN_ERR_UNSUPPORTED
 
 
+def _ws_expected(BH, Nq, d):
+    # dQ accumulator padded to whole 128-row query tiles, D and -log2(e) LSE,
+    # then (16-byte aligned) one int32 order counter per (b*h, query tile).
+    tiles = -(-Nq // 128)
+    words = (BH * Nq + tiles * 128 - Nq) * d + 2 * BH * Nq
+    words = -(-words // 4) * 4
+    return 4 * (words + BH * tiles)
+
+
 def test_workspace_size(lib):
-    assert native.attn_bwd_workspace_bytes(2, 16, 4096, 4096, 64) == 4 * 2 * 16 * 4096 * (64 + 2)
-    assert native.attn_bwd_workspace_bytes(1, 16, 16384, 16384, 128) == 4 * 16 * 16384 * 130
+    assert native.attn_bwd_workspace_bytes(2, 16, 4096, 4096, 64) == 4 * 2 * 16 * 4096 * (64 + 2) + 4 * 32 * 32
+    assert native.attn_bwd_workspace_bytes(1, 16, 16384, 16384, 128) == 4 * 16 * 16384 * 130 + 4 * 16 * 128
     assert native.attn_bwd_workspace_bytes(0, 1, 128, 128, 64) == 0
     assert native.attn_bwd_workspace_bytes(1, 1, -1, 128, 64) == 0
     # A ragged last query tile pads the dQ accumulator to a whole tile.
-    assert native.attn_bwd_workspace_bytes(2, 3, 300, 77, 64) == 4 * ((6 * 300 + 84) * 64 + 2 * 6 * 300)
-    assert native.attn_bwd_workspace_bytes(1, 1, 1, 1, 128) == 4 * (128 * 128 + 2)
+    assert native.attn_bwd_workspace_bytes(2, 3, 300, 77, 64) == _ws_expected(6, 300, 64)
+    assert native.attn_bwd_workspace_bytes(2, 3, 300, 77, 64) >= 4 * ((6 * 300 + 84) * 64 + 2 * 6 * 300)
+    assert native.attn_bwd_workspace_bytes(1, 1, 1, 1, 128) == _ws_expected(1, 1, 128)
+    assert native.attn_bwd_workspace_bytes(3, 1, 5, 9, 64) == _ws_expected(3, 5, 64)
+
+
+@pytest.mark.parametrize("field", ["q", "dq", "workspace"])
+def test_deterministic_bwd_validates_like_bwd(lib, field):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, workspace=FAKE,
+                B=1, H=1, Nq=128, Nk=128, d=64, scale=0.125, causal=0, dtype=native.ATTN_FP16, stream=None)
+    assert native.attn_bwd_deterministic(**{**args, field: None}) == native.ATTN_ERR_INVALID_ARG
+    assert native.attn_bwd_deterministic(**{**args, "d": 96}) == native.ATTN_ERR_UNSUPPORTED
+    assert native.attn_bwd_deterministic(**{**args, "causal": 5}) == native.ATTN_ERR_INVALID_ARG
+    assert native.attn_bwd_deterministic(**{**args, "B": 0}) == native.ATTN_OK
 
 
 def test_tensor_wrapper_rejects_cpu_tensors(lib):

@@ -158,3 +158,46 @@ def test_long_context_workload_windows_and_identities():
         gk, gv, gdo = parity.f64(dkf[s]), parity.f64(dvf[s]), parity.f64(dof[s])
         assert np.linalg.norm(gk.sum(0)) <= parity.GRAD_TOL * np.linalg.norm(gk), tag + " sum dK"
         assert np.linalg.norm(gv.sum(0) - gdo.sum(0)) <= parity.GRAD_TOL * np.linalg.norm(gv), tag + " sum dV"
+
+
+# ------------------------------------------------------- deterministic mode
+
+def run_bwd_det(q, k, v, do, causal, scale, deterministic):
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = native.forward(qd, kd, vd, causal=causal, scale=scale)
+    dq, dk, dv = native.backward(qd, kd, vd, o, lse, dod, causal=causal, scale=scale, deterministic=deterministic)
+    torch.cuda.synchronize()
+    native.device_status()
+    return dq.cpu(), dk.cpu(), dv.cpu()
+
+
+@pytest.mark.parametrize("causal", [False, True, "bottom_right"])
+@pytest.mark.parametrize("dtype,d,nq,nk", [(torch.bfloat16, 128, 640, 640), (torch.float16, 64, 300, 777),
+                                           (torch.bfloat16, 64, 777, 300)])
+def test_deterministic_backward_parity(causal, dtype, d, nq, nk):
+    q, k, v, do = draw(1, 2, nq, nk, d, dtype, seed=61 + nq + d, with_grad=True)
+    dq, dk, dv = run_bwd_det(q, k, v, do, causal, 1 / math.sqrt(d), True)
+    B, H = 1, 2
+    for s in range(B * H):
+        args = [parity.f64(t.reshape(B * H, t.shape[2], d)[s]) for t in (q, k, v, do)]
+        oc, off = parity.oracle_mask(causal, nq, nk)
+        rdq, rdk, rdv = oracle.backward(*args, 1 / math.sqrt(d), oc, off)
+        tag = f"deterministic {dtype} d{d} Nq{nq} Nk{nk} causal={causal} slice {s}"
+        parity.assert_grad(parity.f64(dq.reshape(B * H, nq, d)[s]), rdq, "dQ", tag)
+        parity.assert_grad(parity.f64(dk.reshape(B * H, nk, d)[s]), rdk, "dK", tag)
+        parity.assert_grad(parity.f64(dv.reshape(B * H, nk, d)[s]), rdv, "dV", tag)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_deterministic_backward_is_bit_reproducible(causal):
+    """Many key tiles reduce into each query tile (N = 2048: up to 16), and
+    the grid is larger than the GPU, so atomics would reorder between runs."""
+    q, k, v, do = draw(2, 16, 2048, 2048, 128, torch.bfloat16, seed=67, with_grad=True)
+    runs = [run_bwd_det(q, k, v, do, causal, 1 / math.sqrt(128), True) for _ in range(3)]
+    for r in runs[1:]:
+        for a, b in zip(runs[0], r):
+            assert torch.equal(a, b)
+    # and it agrees with the atomic-order backward to within rounding
+    ref = run_bwd_det(q, k, v, do, causal, 1 / math.sqrt(128), False)
+    for a, b in zip(runs[0], ref):
+        assert parity.rel_fro(parity.f64(a), parity.f64(b)) < 1e-2
