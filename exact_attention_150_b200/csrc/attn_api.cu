@@ -60,14 +60,6 @@ int tiles(int n) { return (n + kTile - 1) / kTile; }
 // the last slice they land here.
 long long pad_rows(int Nq) { return static_cast<long long>(tiles(Nq)) * kTile - Nq; }
 
-// Workspace layout: dQ accumulator [(B*H*Nq + pad_rows) * d] | D [B*H*Nq] |
-// -log2(e) LSE [B*H*Nq] | (16-byte aligned) order counters [B*H][tiles(Nq)]
-// of the deterministic backward.
-long long counters_offset_floats(int BH, int Nq, int d) {
-  const long long rows = static_cast<long long>(BH) * Nq;
-  const long long f = (rows + pad_rows(Nq)) * d + 2 * rows;
-  return (f + 3) / 4 * 4;
-}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -90,30 +82,114 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+// A launch's problems.  Dense batches: one tensor-map slab per (batch,
+// head), all of its rows.  Packed variable-length batches: one slab per
+// head; problem b*H + h is sequence b of head h, whose rows the kernels take
+// from the device offsets cu_q / cu_k.
+struct Problem {
+  int slabs;               // slab count of the tensor maps
+  int rows_q, rows_k;      // rows per slab
+  int problems;            // grid x: B*H
+  int qtiles, ktiles;      // grid y: tiles of the longest query / key sequence
+  const int* cu_q = nullptr;
+  const int* cu_k = nullptr;
+  int H = 1;
+  int bottom_right = 0;
+  bool packed = false;     // variable-length batch
+};
+
+Problem dense_problem(int B, int H, int Nq, int Nk, int causal) {
+  Problem p;
+  p.slabs = p.problems = B * H;
+  p.rows_q = Nq;
+  p.rows_k = Nk;
+  p.qtiles = tiles(Nq);
+  p.ktiles = tiles(Nk);
+  p.bottom_right = causal == ATTN_CAUSAL_BOTTOM_RIGHT;
+  return p;
+}
+
+// Packed variable-length batches: sizes may be zero, not negative; the
+// offsets themselves live on the device and are clamped by the kernels.
+attn_status check_varlen(int B, int H, int total_q, int total_k, int max_q, int max_k, int d, int causal,
+                         attn_dtype dtype) {
+  if (B < 0 || H < 0 || total_q < 0 || total_k < 0 || max_q < 0 || max_k < 0 || d < 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != ATTN_CAUSAL_NONE && causal != ATTN_CAUSAL_TOP_LEFT && causal != ATTN_CAUSAL_BOTTOM_RIGHT)
+    return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_FP16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh > 0x7fffffffLL || tiles(max_q) > 65535 || tiles(max_k) > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(H) * total_q > (1LL << 40) || static_cast<long long>(H) * total_k > (1LL << 40))
+    return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+Problem varlen_problem(int B, int H, int total_q, int total_k, int max_q, int max_k, const int* cu_q,
+                       const int* cu_k, int causal) {
+  Problem p;
+  p.slabs = H;
+  p.rows_q = total_q;
+  p.rows_k = total_k;
+  p.problems = B * H;
+  p.qtiles = tiles(max_q);
+  p.ktiles = tiles(max_k);
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.H = H;
+  p.bottom_right = causal == ATTN_CAUSAL_BOTTOM_RIGHT;
+  p.packed = true;
+  return p;
+}
+
+// Backward workspace of a problem, in 4-byte words: dQ accumulator
+// [(rows + pad) * d] | D [rows] | -log2(e) LSE [rows] | (16-byte aligned)
+// order counters [problems][qtiles] of the deterministic backward, with
+// rows = slabs * rows_q.  The pad takes the reductions of the ragged last
+// query tile's masked rows (exact zeros; see pad_rows); in a packed batch
+// any sequence's last tile can reach up to 127 rows past the total.
+struct WsLayout {
+  long long rows, dvec, nlse2, counters, ncounters, words;
+};
+
+WsLayout ws_layout(const Problem& pb, int d) {
+  WsLayout w;
+  w.rows = static_cast<long long>(pb.slabs) * pb.rows_q;
+  const long long pad = pb.packed ? kTile : pad_rows(pb.rows_q);
+  w.dvec = (w.rows + pad) * d;
+  w.nlse2 = w.dvec + w.rows;
+  w.counters = (w.nlse2 + w.rows + 3) / 4 * 4;
+  w.ncounters = static_cast<long long>(pb.problems) * pb.qtiles;
+  w.words = w.counters + w.ncounters;
+  return w;
+}
+
 template <int D, bool BF16, bool CAUSAL>
 attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse,
-                       int BH, int Nq, int Nk, int off, float scale_log2, cudaStream_t st) {
+                       const Problem& pb, float scale_log2, cudaStream_t st) {
   using L = attn::FwdLayout<D>;
   auto kern = attn::fwd_kernel<D, BF16, CAUSAL>;
   if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
-  dim3 grid(BH, tiles(Nq));
-  kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, Nq, Nk, off, scale_log2);
+  dim3 grid(pb.problems, pb.qtiles);
+  kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, pb.cu_q, pb.cu_k, pb.H, pb.rows_q,
+                                     pb.rows_k, pb.bottom_right, scale_log2);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <int D, bool BF16, bool CAUSAL, bool DET>
 attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                        const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv, float* ws,
-                       int BH, int Nq, int Nk, int off, float scale, int phase, cudaStream_t st) {
+                       const Problem& pb, float scale, int phase, cudaStream_t st) {
   using L = attn::BwdLayout<D>;
-  const long long qrows = static_cast<long long>(BH) * Nq;
+  const WsLayout w = ws_layout(pb, D);
+  const long long qrows = w.rows;
   float* dqacc = ws;
-  float* dvec = ws + (qrows + pad_rows(Nq)) * D;
-  float* nlse2 = dvec + qrows;
-  int* dq_order = DET ? reinterpret_cast<int*>(ws + counters_offset_floats(BH, Nq, D)) : nullptr;
+  float* dvec = ws + w.dvec;
+  float* nlse2 = ws + w.nlse2;
+  int* dq_order = DET ? reinterpret_cast<int*>(ws + w.counters) : nullptr;
 
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_PREPROCESS) {
-    if (DET && cudaMemsetAsync(dq_order, 0, static_cast<size_t>(BH) * tiles(Nq) * sizeof(int), st) != cudaSuccess)
+    if (DET && cudaMemsetAsync(dq_order, 0, static_cast<size_t>(w.ncounters) * sizeof(int), st) != cudaSuccess)
       return ATTN_ERR_CUDA;
     constexpr int kRowsPerBlock = 256 / (D / 8);
     const long long pre_blocks = (qrows + kRowsPerBlock - 1) / kRowsPerBlock;
@@ -124,10 +200,10 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_MAIN) {
     auto kern = attn::bwd_main_kernel<D, BF16, CAUSAL, DET>;
     if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
-    dim3 grid(BH, tiles(Nk));
+    dim3 grid(pb.problems, pb.ktiles);
     kern<<<grid, 512, L::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, dqacc, static_cast<uint16_t*>(dk),
-                                       static_cast<uint16_t*>(dv), dq_order, Nq, Nk, off, scale,
-                                       scale * 1.4426950408889634f);
+                                       static_cast<uint16_t*>(dv), dq_order, pb.cu_q, pb.cu_k, pb.H, pb.rows_q,
+                                       pb.rows_k, pb.bottom_right, pb.qtiles, scale, scale * 1.4426950408889634f);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_CONVERT) {
@@ -141,31 +217,62 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   return ATTN_OK;
 }
 
-// Diagonal offset of the causal mask: query i sees key k iff k <= i + off.
-int causal_offset(int causal, int Nq, int Nk) { return causal == ATTN_CAUSAL_BOTTOM_RIGHT ? Nk - Nq : 0; }
 
 template <int D, bool BF16>
 attn_status dispatch_fwd_causal(int causal, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                                void* o, float* lse, int BH, int Nq, int Nk, float sl2, cudaStream_t st) {
-  const int off = causal_offset(causal, Nq, Nk);
-  return causal ? launch_fwd<D, BF16, true>(mq, mk, mv, o, lse, BH, Nq, Nk, off, sl2, st)
-                : launch_fwd<D, BF16, false>(mq, mk, mv, o, lse, BH, Nq, Nk, off, sl2, st);
+                                void* o, float* lse, const Problem& pb, float sl2, cudaStream_t st) {
+  return causal ? launch_fwd<D, BF16, true>(mq, mk, mv, o, lse, pb, sl2, st)
+                : launch_fwd<D, BF16, false>(mq, mk, mv, o, lse, pb, sl2, st);
+}
+
+// The forward launch shared by attn_fwd and attn_fwd_varlen.
+attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const Problem& pb, int d,
+                     float scale, int causal, attn_dtype dtype, void* stream) {
+  const bool bf16 = dtype == ATTN_BF16;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, pb.slabs, pb.rows_q, d, bf16) || !make_map(&mk, k, pb.slabs, pb.rows_k, d, bf16) ||
+      !make_map(&mv, v, pb.slabs, pb.rows_k, d, bf16))
+    return ATTN_ERR_CUDA;
+  const float sl2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return bf16 ? dispatch_fwd_causal<64, true>(causal, mq, mk, mv, o, lse, pb, sl2, st)
+                : dispatch_fwd_causal<64, false>(causal, mq, mk, mv, o, lse, pb, sl2, st);
+  return bf16 ? dispatch_fwd_causal<128, true>(causal, mq, mk, mv, o, lse, pb, sl2, st)
+              : dispatch_fwd_causal<128, false>(causal, mq, mk, mv, o, lse, pb, sl2, st);
 }
 
 template <int D, bool BF16>
 attn_status dispatch_bwd_causal(int causal, bool det, const CUtensorMap& mq, const CUtensorMap& mk,
                                 const CUtensorMap& mv, const CUtensorMap& mdo, const void* o, const void* dout,
-                                const float* lse, void* dq, void* dk, void* dv, float* ws, int BH, int Nq, int Nk,
+                                const float* lse, void* dq, void* dk, void* dv, float* ws, const Problem& pb,
                                 float scale, int phase, cudaStream_t st) {
-  const int off = causal_offset(causal, Nq, Nk);
 #define ATTN_LAUNCH_BWD(C, DT) \
-  launch_bwd<D, BF16, C, DT>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, off, scale, phase, st)
+  launch_bwd<D, BF16, C, DT>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, pb, scale, phase, st)
   if (det) return causal ? ATTN_LAUNCH_BWD(true, true) : ATTN_LAUNCH_BWD(false, true);
   return causal ? ATTN_LAUNCH_BWD(true, false) : ATTN_LAUNCH_BWD(false, false);
 #undef ATTN_LAUNCH_BWD
 }
 
-// The backward phases shared by attn_bwd_phase (det = false) and
+// The backward launch shared by the dense and packed entry points.
+attn_status bwd_launch(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, void* workspace, const Problem& pb, int d,
+                       float scale, int causal, attn_dtype dtype, int phase, bool det, void* stream) {
+  const bool bf16 = dtype == ATTN_BF16;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, pb.slabs, pb.rows_q, d, bf16) || !make_map(&mk, k, pb.slabs, pb.rows_k, d, bf16) ||
+      !make_map(&mv, v, pb.slabs, pb.rows_k, d, bf16) || !make_map(&mdo, dout, pb.slabs, pb.rows_q, d, bf16))
+    return ATTN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+#define ATTN_DISPATCH_BWD(DD, BB) \
+  dispatch_bwd_causal<DD, BB>(causal, det, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, pb, scale, phase, st)
+  if (d == 64) return bf16 ? ATTN_DISPATCH_BWD(64, true) : ATTN_DISPATCH_BWD(64, false);
+  return bf16 ? ATTN_DISPATCH_BWD(128, true) : ATTN_DISPATCH_BWD(128, false);
+#undef ATTN_DISPATCH_BWD
+}
+
+// The dense backward shared by attn_bwd_phase (det = false) and
 // attn_bwd_deterministic (det = true).
 attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                      void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
@@ -220,27 +327,78 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return ATTN_ERR_INVALID_ARG;
-  const bool bf16 = dtype == ATTN_BF16;
-  const int BH = B * H;
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, BH, Nq, d, bf16) || !make_map(&mk, k, BH, Nk, d, bf16) || !make_map(&mv, v, BH, Nk, d, bf16))
-    return ATTN_ERR_CUDA;
-  const float sl2 = scale * 1.4426950408889634f;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 64)
-    return bf16 ? dispatch_fwd_causal<64, true>(causal, mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st)
-                : dispatch_fwd_causal<64, false>(causal, mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st);
-  return bf16 ? dispatch_fwd_causal<128, true>(causal, mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st)
-              : dispatch_fwd_causal<128, false>(causal, mq, mk, mv, o, lse, BH, Nq, Nk, sl2, st);
+  return fwd_impl(q, k, v, o, lse, dense_problem(B, H, Nq, Nk, causal), d, scale, causal, dtype, stream);
+}
+
+attn_status attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
+                            const int* cu_seqlens_k, int B, int H, int total_q, int total_k, int max_seqlen_q,
+                            int max_seqlen_k, int d, float scale, int causal, attn_dtype dtype, void* stream) {
+  const attn_status cs = check_varlen(B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, d, causal, dtype);
+  if (cs != ATTN_OK) return cs;
+  if (B == 0 || H == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;  // no query rows
+  if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (total_k == 0) {  // no sequence has keys: every row's softmax is empty (O = 0, LSE = -inf)
+    // The kernels write exactly that when they find no key tile; they need a
+    // valid K/V map, so give them the query tensor as a stand-in of one row.
+    return fwd_impl(q, q, q, o, lse, varlen_problem(B, H, total_q, 1, max_seqlen_q, 1, cu_seqlens_q, cu_seqlens_k,
+                                                    causal), d, scale, causal, dtype, stream);
+  }
+  return fwd_impl(q, k, v, o, lse,
+                  varlen_problem(B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, cu_seqlens_q, cu_seqlens_k,
+                                 causal),
+                  d, scale, causal, dtype, stream);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
   if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return 0;  // empty problems need none
   const long long bh = static_cast<long long>(B) * H;
   if (bh > 0x7fffffffLL || bh * Nq > (1LL << 40)) return 0;
-  const unsigned long long words = static_cast<unsigned long long>(counters_offset_floats(static_cast<int>(bh), Nq, d)) +
-                                   static_cast<unsigned long long>(bh) * tiles(Nq);
-  return static_cast<size_t>(words * 4);
+  return static_cast<size_t>(ws_layout(dense_problem(B, H, Nq, Nk, 0), d).words * 4);
+}
+
+size_t attn_bwd_varlen_workspace_bytes(int B, int H, int total_q, int max_seqlen_q, int d) {
+  if (B <= 0 || H <= 0 || total_q <= 0 || max_seqlen_q <= 0 || d <= 0) return 0;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL || static_cast<long long>(H) * total_q > (1LL << 40)) return 0;
+  return static_cast<size_t>(
+      ws_layout(varlen_problem(B, H, total_q, 1, max_seqlen_q, 1, nullptr, nullptr, 0), d).words * 4);
+}
+
+attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dout, void* dq, void* dk, void* dv, void* workspace, const int* cu_seqlens_q,
+                            const int* cu_seqlens_k, int B, int H, int total_q, int total_k, int max_seqlen_q,
+                            int max_seqlen_k, int d, float scale, int causal, attn_dtype dtype, int deterministic,
+                            void* stream) {
+  const attn_status cs = check_varlen(B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, d, causal, dtype);
+  if (cs != ATTN_OK) return cs;
+  if (B == 0 || H == 0) return ATTN_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (total_q == 0 || max_seqlen_q == 0) {  // no query rows: dK = dV = 0
+    const size_t bytes = static_cast<size_t>(H) * total_k * d * 2;
+    if (bytes == 0) return ATTN_OK;
+    if (!dk || !dv) return ATTN_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(dk, 0, bytes, st) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, st) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    return ATTN_OK;
+  }
+  if (total_k == 0) {  // no key rows: every softmax is empty, so dQ = 0
+    if (!dq) return ATTN_ERR_INVALID_ARG;
+    return cudaMemsetAsync(dq, 0, static_cast<size_t>(H) * total_q * d * 2, st) == cudaSuccess ? ATTN_OK
+                                                                                                 : ATTN_ERR_CUDA;
+  }
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace || !cu_seqlens_q || !cu_seqlens_k)
+    return ATTN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  return bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace,
+                    varlen_problem(B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, cu_seqlens_q, cu_seqlens_k,
+                                   causal),
+                    d, scale, causal, dtype, ATTN_BWD_ALL, deterministic != 0, stream);
 }
 
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
@@ -290,19 +448,8 @@ attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
   const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
   for (const void* p : ptrs)
     if (!aligned16(p)) return ATTN_ERR_INVALID_ARG;
-  const bool bf16 = dtype == ATTN_BF16;
-  const int BH = B * H;
-  CUtensorMap mq, mk, mv, mdo;
-  if (!make_map(&mq, q, BH, Nq, d, bf16) || !make_map(&mk, k, BH, Nk, d, bf16) ||
-      !make_map(&mv, v, BH, Nk, d, bf16) || !make_map(&mdo, dout, BH, Nq, d, bf16))
-    return ATTN_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* ws = static_cast<float*>(workspace);
-#define ATTN_DISPATCH_BWD(DD, BB) \
-  dispatch_bwd_causal<DD, BB>(causal, det, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, BH, Nq, Nk, scale, phase, st)
-  if (d == 64) return bf16 ? ATTN_DISPATCH_BWD(64, true) : ATTN_DISPATCH_BWD(64, false);
-  return bf16 ? ATTN_DISPATCH_BWD(128, true) : ATTN_DISPATCH_BWD(128, false);
-#undef ATTN_DISPATCH_BWD
+  return bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, dense_problem(B, H, Nq, Nk, causal), d, scale,
+                    causal, dtype, phase, det, stream);
 }
 
 }  // namespace

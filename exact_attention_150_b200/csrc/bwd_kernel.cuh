@@ -167,7 +167,8 @@ __global__ void __launch_bounds__(512, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const float* __restrict__ dvec, const float* __restrict__ nlse2, float* __restrict__ dqacc,
                     uint16_t* __restrict__ dk_ptr, uint16_t* __restrict__ dv_ptr, int* __restrict__ dq_order,
-                    int Nq, int Nk, int off, float scale, float scale_log2) {
+                    const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H, int Nq, int Nk,
+                    int bottom_right, int order_stride, float scale, float scale_log2) {
   using L = BwdLayout<D>;
   constexpr bool kDqT = (D == 128);  // dQ formed transposed (see above)
   constexpr uint32_t kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 256 + D;
@@ -193,22 +194,44 @@ __global__ void __launch_bounds__(512, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int bh = blockIdx.x;
+  // The problem of this CTA: slab z of the tensor maps ([z][Nq or Nk][D])
+  // and rows [q0, q0 + nq) / [k0, k0 + nk) of it (one slab per (batch,
+  // head) for dense batches; one per head for packed variable-length
+  // batches, sequence b's rows from the offsets clamped to the slab).
+  int z = blockIdx.x, q0 = 0, k0 = 0, nq = Nq, nk = Nk;
+  if (cu_q != nullptr) {
+    const int b = static_cast<int>(blockIdx.x) / H;
+    z = static_cast<int>(blockIdx.x) - b * H;
+    auto clamp = [](int v, int hi) { return v < 0 ? 0 : (v > hi ? hi : v); };
+    q0 = clamp(cu_q[b], Nq);
+    k0 = clamp(cu_k[b], Nk);
+    nq = clamp(cu_q[b + 1], Nq) - q0;
+    nk = clamp(cu_k[b + 1], Nk) - k0;
+    nq = nq < 0 ? 0 : nq;
+    nk = nk < 0 ? 0 : nk;
+    // Rows past max_seqlen_q (the grid's query tiles) are not computed; this
+    // also keeps the order counters of the deterministic mode in range.
+    nq = nq < order_stride * kBwdTile ? nq : order_stride * kBwdTile;
+  }
   const int j = blockIdx.y;  // key tile; causal: small j has the most work and launches first
-  const int nqt = (Nq + kBwdTile - 1) / kBwdTile;  // the last tiles may be ragged
+  if (j * kBwdTile >= nk) return;  // a sequence shorter than the grid
+  const int nqt = (nq + kBwdTile - 1) / kBwdTile;  // the last tiles may be ragged
   // Causal: query q sees key k iff k <= q + off (off = 0 top-left,
-  // Nk - Nq bottom-right); the first query tile that sees key j * 128 is
+  // nk - nq bottom-right); the first query tile that sees key j * 128 is
   // the one holding query j * 128 - off.
+  const int off = bottom_right ? nk - nq : 0;
   const int first_q = j * kBwdTile - off;
   const int i0 = CAUSAL ? (first_q > 0 ? first_q / kBwdTile : 0) : 0;
   const int n_it = nqt - i0;
-  const int kv_valid = Nk - j * kBwdTile < kBwdTile ? Nk - j * kBwdTile : kBwdTile;  // key rows of this tile
+  const int kv_valid = nk - j * kBwdTile < kBwdTile ? nk - j * kBwdTile : kBwdTile;  // key rows of this tile
+  const size_t krow0 = static_cast<size_t>(z) * Nk + k0 + static_cast<size_t>(j) * kBwdTile;  // first key row
+  const size_t qslab = static_cast<size_t>(z) * Nq + q0;  // row of this sequence's first query
 
   if (n_it <= 0) {
-    // Causal with more keys than queries: no query sees these keys, so
-    // their gradients are zero.
+    // No query sees these keys (causal with more keys than queries, or a
+    // sequence without queries): their gradients are zero.
     const int n16 = kv_valid * D / 8;
-    const size_t base = (static_cast<size_t>(bh) * Nk + static_cast<size_t>(j) * kBwdTile) * D / 8;
+    const size_t base = krow0 * D / 8;
     for (int e = threadIdx.x; e < n16; e += blockDim.x) {
       reinterpret_cast<uint4*>(dk_ptr)[base + e] = make_uint4(0u, 0u, 0u, 0u);
       reinterpret_cast<uint4*>(dv_ptr)[base + e] = make_uint4(0u, 0u, 0u, 0u);
@@ -269,8 +292,8 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(kv_full, 2 * L::kTileBytes);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(smem + L::kKOff + c * L::kChunkBytes, &tm_k, kv_full, c * 64, j * kBwdTile, bh);
-        tma_load_3d(smem + L::kVOff + c * L::kChunkBytes, &tm_v, kv_full, c * 64, j * kBwdTile, bh);
+        tma_load_3d(smem + L::kKOff + c * L::kChunkBytes, &tm_k, kv_full, c * 64, k0 + j * kBwdTile, z);
+        tma_load_3d(smem + L::kVOff + c * L::kChunkBytes, &tm_v, kv_full, c * 64, k0 + j * kBwdTile, z);
       }
       int it = 0;
       bool ok = true;
@@ -281,12 +304,12 @@ __global__ void __launch_bounds__(512, 1)
           ok = false;
           break;
         }
-        const int qrow = (i0 + it) * kBwdTile;
+        const int qrow = q0 + (i0 + it) * kBwdTile;
         mbar_arrive_expect_tx(&qd_full[s], 2 * L::kTileBytes);
         uint8_t* qdst = smem + L::kStageOff + s * 2 * L::kTileBytes;
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(qdst + c * L::kChunkBytes, &tm_q, &qd_full[s], c * 64, qrow, bh);
-          tma_load_3d(qdst + L::kTileBytes + c * L::kChunkBytes, &tm_do, &qd_full[s], c * 64, qrow, bh);
+          tma_load_3d(qdst + c * L::kChunkBytes, &tm_q, &qd_full[s], c * 64, qrow, z);
+          tma_load_3d(qdst + L::kTileBytes + c * L::kChunkBytes, &tm_do, &qd_full[s], c * 64, qrow, z);
         }
       }
       if (!ok) {
@@ -418,12 +441,12 @@ __global__ void __launch_bounds__(512, 1)
       return pack2<BF16>(hi, v - hi);
     };
     for (int it = 0; it < n_it; ++it) {
-      const size_t vbase = static_cast<size_t>(bh) * Nq + static_cast<size_t>(i0 + it) * kBwdTile;
-      const int q_valid = Nq - (i0 + it) * kBwdTile;
+      const size_t vbase = qslab + static_cast<size_t>(i0 + it) * kBwdTile;
+      const int q_valid = nq - (i0 + it) * kBwdTile;
       float sv[4], dv4[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const bool in = lane + 32 * k < q_valid;  // rows past Nq: zeros (their P is masked)
+        const bool in = lane + 32 * k < q_valid;  // rows past the sequence: zeros (their P is masked)
         sv[k] = in ? nlse2[vbase + lane + 32 * k] * inv_c : 0.f;
         dv4[k] = in ? -dvec[vbase + lane + 32 * k] : 0.f;
       }
@@ -451,7 +474,7 @@ __global__ void __launch_bounds__(512, 1)
       // Key row r sees query columns [lo, hi) of this tile: lo from the
       // causal mask, hi = the queries before Nq, and none at all if the key
       // is past Nk.  P is zeroed outside.
-      const int q_valid = Nq - i * kBwdTile;
+      const int q_valid = nq - i * kBwdTile;
       const bool masked = diag || kv_valid < kBwdTile || q_valid < kBwdTile;
       const int lo = diag && dlt + r > 0 ? dlt + r : 0;
       const int hi = r < kv_valid ? (q_valid < kBwdTile ? q_valid : kBwdTile) : 0;
@@ -534,13 +557,13 @@ __global__ void __launch_bounds__(512, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const size_t qrow0 = static_cast<size_t>(bh) * Nq + static_cast<size_t>(i0 + it) * kBwdTile;
+      const size_t qrow0 = qslab + static_cast<size_t>(i0 + it) * kBwdTile;
       // Deterministic mode: the key tiles that reach a query tile are a
       // prefix 0..J of the key tiles (the first query tile a key tile sees
       // never decreases with it), so this CTA is contributor number j of
       // every query tile it covers.  It reduces into the tile only after the
       // 4 drain warps of contributors 0..j-1 have each counted theirs.
-      int* turn = DET ? dq_order + static_cast<size_t>(bh) * nqt + (i0 + it) : nullptr;
+      int* turn = DET ? dq_order + static_cast<size_t>(blockIdx.x) * order_stride + (i0 + it) : nullptr;
       auto await_turn = [&]() {
         if constexpr (DET) {
           if (!__all_sync(0xffffffffu, wait_turn(turn, 4 * j, abort_flag))) return false;
@@ -563,7 +586,7 @@ __global__ void __launch_bounds__(512, 1)
         // d of one query row (128 contiguous bytes).
         // All 128 columns are read before the columns are released, so the
         // next dP^T product does not wait for the reductions.  Query rows
-        // past Nq in a ragged tile hold exact zeros (masked P) and are
+        // past the sequence in a ragged tile hold exact zeros (masked P) and are
         // reduced like the others; the host pads the accumulator for them.
         float* base = dqacc + qrow0 * D + row;
         uint32_t va[32], vb[32], vc[32], vd[32];
@@ -615,7 +638,7 @@ __global__ void __launch_bounds__(512, 1)
       if (__all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag))) {
         tc_fence_after();
         // dK / dV: M = keys, so the TMEM lane is the key row.
-        const size_t grow = static_cast<size_t>(bh) * Nk + static_cast<size_t>(j) * kBwdTile + row;
+        const size_t grow = krow0 + row;
         const bool live = row < kv_valid;  // padding rows of a ragged key tile are not stored
         uint4* dvd = reinterpret_cast<uint4*>(dv_ptr + grow * D);
         uint4* dkd = reinterpret_cast<uint4*>(dk_ptr + grow * D);

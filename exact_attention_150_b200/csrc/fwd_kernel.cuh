@@ -80,7 +80,8 @@ template <int D, bool BF16, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o_ptr,
-               float* __restrict__ lse_ptr, int Nq, int Nk, int off, float scale_log2) {
+               float* __restrict__ lse_ptr, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H,
+               int Nq, int Nk, int bottom_right, float scale_log2) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -104,24 +105,43 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int bh = blockIdx.x;
-  const int nqt = (Nq + kTile - 1) / kTile;  // the last tiles may be ragged
-  const int nkt = (Nk + kTile - 1) / kTile;
+  // The problem of this CTA: slab z of the tensor maps ([z][Nq or Nk][D])
+  // and rows [q0, q0 + nq) / [k0, k0 + nk) of it.  Dense batches have one
+  // slab per (batch, head) and use all of it.  Packed variable-length
+  // batches have one slab per head and take sequence b's rows from the
+  // offsets, clamped to the slab: bad offsets can give wrong values but
+  // never address outside the tensors.
+  int z = blockIdx.x, q0 = 0, k0 = 0, nq = Nq, nk = Nk;
+  if (cu_q != nullptr) {
+    const int b = static_cast<int>(blockIdx.x) / H;
+    z = static_cast<int>(blockIdx.x) - b * H;
+    auto clamp = [](int v, int hi) { return v < 0 ? 0 : (v > hi ? hi : v); };
+    q0 = clamp(cu_q[b], Nq);
+    k0 = clamp(cu_k[b], Nk);
+    nq = clamp(cu_q[b + 1], Nq) - q0;
+    nk = clamp(cu_k[b + 1], Nk) - k0;
+    nq = nq < 0 ? 0 : nq;
+    nk = nk < 0 ? 0 : nk;
+  }
+  const int nqt = (nq + kTile - 1) / kTile;  // the last tiles may be ragged
+  const int nkt = (nk + kTile - 1) / kTile;
+  if (static_cast<int>(blockIdx.y) >= nqt) return;  // a sequence shorter than the grid
   // Causal: the heaviest query tiles are launched first.
   const int qt = CAUSAL ? (nqt - 1 - static_cast<int>(blockIdx.y)) : static_cast<int>(blockIdx.y);
   // Key tiles this query tile sees.  Causal: query i sees key k iff
-  // k <= i + off (off = 0 top-left, Nk - Nq bottom-right).
+  // k <= i + off (off = 0 top-left, nk - nq bottom-right).
+  const int off = bottom_right ? nk - nq : 0;
   int n = nkt;
   if (CAUSAL) {
-    const int last_row = qt * kTile + kTile - 1 < Nq - 1 ? qt * kTile + kTile - 1 : Nq - 1;
-    const int last_key = last_row + off < Nk - 1 ? last_row + off : Nk - 1;
+    const int last_row = qt * kTile + kTile - 1 < nq - 1 ? qt * kTile + kTile - 1 : nq - 1;
+    const int last_key = last_row + off < nk - 1 ? last_row + off : nk - 1;
     n = last_key < 0 ? 0 : last_key / kTile + 1;
   }
   if (n == 0) {
-    // No row of this tile sees a key (bottom-right with Nq > Nk): the
-    // softmax is empty, O = 0 and LSE = log 0.
-    const int rows = Nq - qt * kTile < kTile ? Nq - qt * kTile : kTile;
-    const size_t grow0 = static_cast<size_t>(bh) * Nq + static_cast<size_t>(qt) * kTile;
+    // No row of this tile sees a key (bottom-right with nq > nk, or a
+    // sequence without keys): the softmax is empty, O = 0 and LSE = log 0.
+    const int rows = nq - qt * kTile < kTile ? nq - qt * kTile : kTile;
+    const size_t grow0 = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile;
     for (int e = threadIdx.x; e < rows * D / 8; e += blockDim.x)
       reinterpret_cast<uint4*>(o_ptr + grow0 * D)[e] = make_uint4(0u, 0u, 0u, 0u);
     for (int e = threadIdx.x; e < rows; e += blockDim.x) lse_ptr[grow0 + e] = -INFINITY;
@@ -177,7 +197,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(q_full, L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
-        tma_load_3d(smem + L::kQOff + c * L::kChunkBytes, &tm_q, q_full, c * 64, qt * kTile, bh);
+        tma_load_3d(smem + L::kQOff + c * L::kChunkBytes, &tm_q, q_full, c * 64, q0 + qt * kTile, z);
       // Ring order: K_0, K_1, then V_j, K_{j+2} for j = 0, 1, ...
       int item = 0;
       bool ok = true;
@@ -187,7 +207,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
         uint8_t* dst = smem + L::kRingOff + slot * L::kTileBytes;
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * 64, tile * kTile, bh);
+          tma_load_3d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * 64, k0 + tile * kTile, z);
         ++item;
         return true;
       };
@@ -225,8 +245,8 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t kd = sdesc_sw128(k_addr, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-        mma_ts(tmem + L::kColS + 128 * b, tmem + L::kColQ + 8 * ks, kd + (off >> 4), kIdS, ks > 0 ? 1u : 0u);
+        const uint32_t step = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
+        mma_ts(tmem + L::kColS + 128 * b, tmem + L::kColQ + 8 * ks, kd + (step >> 4), kIdS, ks > 0 ? 1u : 0u);
       }
     };
     // O += P V: P in the buffer's TMEM columns (key step ks of 16 keys sits
@@ -340,9 +360,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 64; ++c) x[c] *= scale_log2;
       }
-      // Mask keys past Nk (ragged last tile) and, causal, keys after
+      // Mask keys past nk (ragged last tile) and, causal, keys after
       // query + off: column c is kept iff c <= lim.
-      const int kv_valid = Nk - j * kTile;
+      const int kv_valid = nk - j * kTile;
       const int diag_lim = (qt - j) * kTile + off;  // lim of row 0 from the mask
       if ((CAUSAL && diag_lim < kTile - 1) || kv_valid < kTile) {
         int lim = kv_valid - 1;
@@ -451,8 +471,8 @@ __global__ void __launch_bounds__(384, 1)
       const bool empty = m_run == -INFINITY;
       const float l_tc = __uint_as_float(tmem_ld1(t_row + L::kColL));
       const float inv = empty ? 0.f : 1.f / l_tc;
-      const bool live = qt * kTile + row < Nq;  // padding rows of a ragged tile are not stored
-      const size_t grow = static_cast<size_t>(bh) * Nq + static_cast<size_t>(qt) * kTile + row;
+      const bool live = qt * kTile + row < nq;  // padding rows of a ragged tile are not stored
+      const size_t grow = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile + row;
       uint4* dst = reinterpret_cast<uint4*>(o_ptr + grow * D + (D / 2) * h);
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {

@@ -53,6 +53,13 @@ def load() -> ctypes.CDLL:
     lib.attn_bwd_phase.restype = st
     lib.attn_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
     lib.attn_bwd_deterministic.restype = st
+    lib.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, vp]
+    lib.attn_fwd_varlen.restype = st
+    lib.attn_bwd_varlen_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.attn_bwd_varlen_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i,
+                                    vp]
+    lib.attn_bwd_varlen.restype = st
     lib.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
     lib.attn_bwd_noalloc.restype = st
     lib.attn_bwd_noalloc_max_scratch_bytes.argtypes = []
@@ -220,6 +227,94 @@ def backward(q, k, v, out, lse, dout, causal=False, scale: float | None = None,
     else:
         _check("attn_bwd", attn_bwd_phase(*ptrs, B, H, Nq, Nk, d, float(scale), causal_code(causal), code, phase,
                                           stream))
+    return dq, dk, dv
+
+
+# ------------------------------------------------ packed variable-length
+
+def attn_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, total_q, total_k, max_q, max_k, d, scale, causal, dtype,
+                    stream) -> int:
+    """Direct call of attn_fwd_varlen with integer device pointers."""
+    return load().attn_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, total_q, total_k, max_q, max_k, d, scale,
+                                  int(causal), dtype, stream)
+
+
+def attn_bwd_varlen_workspace_bytes(B, H, total_q, max_q, d) -> int:
+    return int(load().attn_bwd_varlen_workspace_bytes(B, H, total_q, max_q, d))
+
+
+def attn_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_q, cu_k, B, H, total_q, total_k, max_q, max_k,
+                    d, scale, causal, dtype, deterministic, stream) -> int:
+    """Direct call of attn_bwd_varlen with integer device pointers."""
+    return load().attn_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_q, cu_k, B, H, total_q, total_k,
+                                  max_q, max_k, d, scale, int(causal), dtype, int(deterministic), stream)
+
+
+def _check_cu(name, cu, B):
+    if not cu.is_cuda or cu.dtype != torch.int32 or tuple(cu.shape) != (B + 1,) or not cu.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA int32 tensor of shape ({B + 1},)")
+
+
+def forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int, causal=False,
+                   scale: float | None = None, out=None, lse=None, stream=None):
+    """O, LSE of a packed variable-length batch: q [H, total_q, d], k and v
+    [H, total_k, d]; sequence b is rows cu_seqlens[b]:cu_seqlens[b+1]."""
+    H, total_q, d = q.shape
+    total_k = k.shape[1]
+    B = cu_seqlens_q.shape[0] - 1
+    code = _dtype_code(q)
+    _check_tensor("q", q, (H, total_q, d), q.dtype)
+    _check_tensor("k", k, (H, total_k, d), q.dtype)
+    _check_tensor("v", v, (H, total_k, d), q.dtype)
+    _check_cu("cu_seqlens_q", cu_seqlens_q, B)
+    _check_cu("cu_seqlens_k", cu_seqlens_k, B)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, (H, total_q, d), q.dtype)
+    _check_tensor("lse", lse, (H, total_q), torch.float32)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    _check("attn_fwd_varlen", attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                              cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, H, total_q,
+                                              total_k, int(max_seqlen_q), int(max_seqlen_k), d, float(scale),
+                                              causal_code(causal), code, stream))
+    return out, lse
+
+
+def backward_varlen(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                    causal=False, scale: float | None = None, dq=None, dk=None, dv=None, workspace=None,
+                    deterministic: bool = False, stream=None):
+    """dQ, dK, dV of forward_varlen for the output gradient dout."""
+    H, total_q, d = q.shape
+    total_k = k.shape[1]
+    B = cu_seqlens_q.shape[0] - 1
+    code = _dtype_code(q)
+    for name, t, shp in (("q", q, (H, total_q, d)), ("k", k, (H, total_k, d)), ("v", v, (H, total_k, d)),
+                         ("out", out, (H, total_q, d)), ("dout", dout, (H, total_q, d))):
+        _check_tensor(name, t, shp, q.dtype)
+    _check_tensor("lse", lse, (H, total_q), torch.float32)
+    _check_cu("cu_seqlens_q", cu_seqlens_q, B)
+    _check_cu("cu_seqlens_k", cu_seqlens_k, B)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = attn_bwd_varlen_workspace_bytes(B, H, total_q, int(max_seqlen_q), d)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    if workspace.numel() * workspace.element_size() < nbytes or not workspace.is_cuda:
+        raise ValueError(f"workspace must be a CUDA buffer of at least {nbytes} bytes")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    _check("attn_bwd_varlen", attn_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                              lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                              dv.data_ptr(), workspace.data_ptr(), cu_seqlens_q.data_ptr(),
+                                              cu_seqlens_k.data_ptr(), B, H, total_q, total_k, int(max_seqlen_q),
+                                              int(max_seqlen_k), d, float(scale), causal_code(causal), code,
+                                              deterministic, stream))
     return dq, dk, dv
 
 

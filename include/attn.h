@@ -205,6 +205,44 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
 size_t attn_bwd_noalloc_max_scratch_bytes(void);
 
 /*
+ * Packed variable-length batches.  B sequences of different lengths share
+ * one tensor without padding (the pages' "varlen" use: each sequence is an
+ * attention problem of its own).  Layout, head-major like the dense calls:
+ * Q, O, dO, dQ are [H][total_q][d]; K, V, dK, dV are [H][total_k][d]; LSE is
+ * [H][total_q].  Sequence b occupies rows [cu_seqlens_q[b], cu_seqlens_q[b+1])
+ * of every head of Q, O, dO, dQ and LSE, and rows [cu_seqlens_k[b],
+ * cu_seqlens_k[b+1]) of every head of K, V, dK, dV.
+ *   cu_seqlens_q, cu_seqlens_k  DEVICE int32 arrays of B + 1 non-decreasing
+ *                offsets from 0 to total_q (total_k), 4-byte aligned.  They
+ *                are read by the kernels and not checked on the host; the
+ *                kernels clamp them to [0, total], so invalid offsets can give
+ *                wrong values but never address memory outside the tensors.
+ *   max_seqlen_q, max_seqlen_k  at least the longest sequence (they size the
+ *                grid; rows of a longer sequence past them are not computed).
+ * The causal mask, top-left or bottom-right, is aligned within each
+ * sequence.  A sequence with queries and no keys gets O = 0, LSE = -inf and
+ * dQ = 0; one with keys and no queries gets dK = dV = 0.  Other arguments,
+ * supported head dims and dtypes, and errors as for the dense calls.
+ */
+attn_status attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H,
+                            int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                            float scale, int causal, attn_dtype dtype, void* stream);
+
+/* Workspace of attn_bwd_varlen, laid out as for attn_bwd with B*H*Nq rows
+ * replaced by H*total_q and 128 padding rows; 0 for an empty batch. */
+size_t attn_bwd_varlen_workspace_bytes(int B, int H, int total_q, int max_seqlen_q, int d);
+
+/* Backward of attn_fwd_varlen; deterministic != 0 orders the dQ reductions
+ * as attn_bwd_deterministic does. */
+attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                            void* workspace, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                            int B, int H, int total_q, int total_k, int max_seqlen_q,
+                            int max_seqlen_k, int d, float scale, int causal, attn_dtype dtype,
+                            int deterministic, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word that
  * kernels of this library set when a bounded wait times out
  * (ATTN_ERR_TIMEOUT), or ATTN_ERR_CUDA if the synchronisation itself fails.

@@ -188,3 +188,43 @@ def test_causal_codes_match_the_header():
     assert [native.causal_code(c) for c in (False, True, "none", "top_left", "bottom_right", 2)] == [0, 1, 0, 1, 2, 2]
     with pytest.raises(ValueError):
         native.causal_code("bottom-left")
+
+
+def _fwd_varlen(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, cu_q=FAKE, cu_k=FAKE, B=2, H=3, total_q=300, total_k=400,
+                max_q=200, max_k=300, d=64, scale=0.125, causal=0, dtype=native.ATTN_BF16, stream=None)
+    args.update(kw)
+    return native.attn_fwd_varlen(**args)
+
+
+def _bwd_varlen(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, workspace=FAKE,
+                cu_q=FAKE, cu_k=FAKE, B=2, H=3, total_q=300, total_k=400, max_q=200, max_k=300, d=64, scale=0.125,
+                causal=0, dtype=native.ATTN_BF16, deterministic=0, stream=None)
+    args.update(kw)
+    return native.attn_bwd_varlen(**args)
+
+
+@pytest.mark.parametrize("fn", [_fwd_varlen, _bwd_varlen])
+def test_varlen_validation(lib, fn):
+    for field in ("B", "H", "total_q", "total_k", "max_q", "max_k"):
+        assert fn(**{field: -1}) == native.ATTN_ERR_INVALID_ARG
+    assert fn(d=96) == native.ATTN_ERR_UNSUPPORTED
+    assert fn(dtype=5) == native.ATTN_ERR_UNSUPPORTED
+    assert fn(causal=3) == native.ATTN_ERR_INVALID_ARG
+    assert fn(max_q=65535 * 128 + 1) == native.ATTN_ERR_UNSUPPORTED
+    assert fn(cu_q=None) == native.ATTN_ERR_INVALID_ARG
+    assert fn(cu_k=FAKE + 2) == native.ATTN_ERR_INVALID_ARG  # offsets must be 4-byte aligned
+    assert fn(q=FAKE + 8) == native.ATTN_ERR_INVALID_ARG
+    assert fn(B=0) == native.ATTN_OK
+    assert fn(H=0) == native.ATTN_OK
+
+
+def test_varlen_workspace_size(lib):
+    for B, H, total_q, max_q, d in ((2, 3, 300, 200, 64), (5, 16, 4096, 1024, 128), (1, 1, 1, 1, 128)):
+        tiles = -(-max_q // 128)
+        rows = H * total_q
+        words = (rows + 128) * d + 2 * rows
+        words = -(-words // 4) * 4 + B * H * tiles
+        assert native.attn_bwd_varlen_workspace_bytes(B, H, total_q, max_q, d) == 4 * words
+    assert native.attn_bwd_varlen_workspace_bytes(0, 3, 300, 200, 64) == 0
