@@ -280,6 +280,37 @@ attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
 
 }  // namespace
 
+// ------------------------------------------------ failure-detection self-test
+
+namespace attn {
+
+// One CTA of 64 threads.  Warp 0 waits, through the attention kernels' own
+// bounded wait, on a barrier that nothing arrives on: it gives up after
+// limit_ns, raises the CTA's abort flag and records the timeout.  Warp 1
+// waits on a second such barrier with the kernels' 1 s limit and leaves
+// through the abort flag as the other roles of an attention kernel would.
+__global__ void __launch_bounds__(64) selftest_wait_kernel(unsigned long long limit_ns, int* result) {
+  __shared__ uint64_t bars[2];
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* abort = &abort_flag;
+  bool ok;
+  if (threadIdx.x < 32)
+    ok = __all_sync(0xffffffffu, mbar_wait_for(&bars[0], 0, abort, limit_ns));
+  else
+    ok = __all_sync(0xffffffffu, mbar_wait(&bars[1], 0, abort));
+  __syncthreads();
+  if (threadIdx.x % 32 == 0) result[threadIdx.x / 32] = ok ? 1 : 0;
+}
+
+}  // namespace attn
+
 // ------------------------------------------------ allocation-free backward
 //
 // attn_bwd_noalloc runs the backward pass with its workspace in this fixed
@@ -476,6 +507,13 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
 }
 
 size_t attn_bwd_noalloc_max_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+attn_status attn_selftest_wait_timeout(int limit_us, int* result, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000 || !result) return ATTN_ERR_INVALID_ARG;
+  attn::selftest_wait_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_us) * 1000ull, result);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
 
 attn_status attn_last_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;

@@ -69,9 +69,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits until the phase of parity `parity` of `bar` has completed.  Returns
-// false (after recording a timeout) if that takes longer than the limit, or as
-// soon as another role of the CTA has raised `abort`.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// false (after raising `abort` and recording a timeout in the device status
+// word) if that takes longer than `limit_ns`, or as soon as another role of
+// the CTA has raised `abort`.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              unsigned long long limit_ns) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = global_ns();
@@ -80,12 +82,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
     if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit_ns) {
       *abort = 1;
       atomicExch(&g_device_status, kStatusTimeout);
       return false;
     }
   }
+}
+
+// The wait every role of the attention kernels uses.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
 // Same wait with a short, fixed limit and no abort check: used on the error

@@ -64,6 +64,8 @@ def load() -> ctypes.CDLL:
     lib.attn_bwd_noalloc.restype = st
     lib.attn_bwd_noalloc_max_scratch_bytes.argtypes = []
     lib.attn_bwd_noalloc_max_scratch_bytes.restype = ctypes.c_size_t
+    lib.attn_selftest_wait_timeout.argtypes = [i, vp, vp]
+    lib.attn_selftest_wait_timeout.restype = st
     lib.attn_last_device_status.argtypes = [vp]
     lib.attn_last_device_status.restype = st
     lib.attn_status_string.argtypes = [st]
@@ -316,6 +318,15 @@ def backward_varlen(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seq
                                               int(max_seqlen_k), d, float(scale), causal_code(causal), code,
                                               deterministic, stream))
     return dq, dk, dv
+
+
+def selftest_wait_timeout(limit_us: int, result, stream=None) -> int:
+    """Launches the failure-detection self-test (see include/attn.h); result
+    is a CUDA int32 tensor of 2 elements.  Returns the launch status."""
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return int(load().attn_selftest_wait_timeout(int(limit_us), result.data_ptr() if result is not None else None,
+                                                  stream))
 
 
 def device_status(stream=None) -> None:

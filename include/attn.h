@@ -243,6 +243,20 @@ attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const v
                             int deterministic, void* stream);
 
 /*
+ * Self-test of failure detection; the paper has no counterpart.  Launches one
+ * small kernel on `stream`.  Its first warp waits, through the same bounded
+ * mbarrier wait the attention kernels use, on a barrier that nothing ever
+ * arrives on, with a limit of `limit_us` microseconds (1 .. 1,000,000).  The
+ * wait gives up, raises the CTA's abort flag and records ATTN_ERR_TIMEOUT in
+ * the device status word.  A second warp, waiting on another such barrier,
+ * leaves through the abort flag.  The kernel then exits normally and the
+ * context stays usable.  result (device, 2 ints) receives 0 for each warp
+ * whose wait gave up.  Returns ATTN_OK once launched; read the status with
+ * attn_last_device_status().
+ */
+attn_status attn_selftest_wait_timeout(int limit_us, int* result, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word that
  * kernels of this library set when a bounded wait times out
  * (ATTN_ERR_TIMEOUT), or ATTN_ERR_CUDA if the synchronisation itself fails.

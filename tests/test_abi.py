@@ -228,3 +228,12 @@ def test_varlen_workspace_size(lib):
         words = -(-words // 4) * 4 + B * H * tiles
         assert native.attn_bwd_varlen_workspace_bytes(B, H, total_q, max_q, d) == 4 * words
     assert native.attn_bwd_varlen_workspace_bytes(0, 3, 300, 200, 64) == 0
+
+
+@pytest.mark.parametrize("limit_us", [0, -5, 1000001])
+def test_selftest_rejects_bad_limits(lib, limit_us):
+    assert native.load().attn_selftest_wait_timeout(limit_us, FAKE, None) == native.ATTN_ERR_INVALID_ARG
+
+
+def test_selftest_rejects_null_result(lib):
+    assert native.load().attn_selftest_wait_timeout(1000, None, None) == native.ATTN_ERR_INVALID_ARG
