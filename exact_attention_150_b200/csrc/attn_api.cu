@@ -69,7 +69,7 @@ attn_status check_common(int B, int H, int Nq, int Nk, int d, int causal, attn_d
   if (causal != ATTN_CAUSAL_NONE && causal != ATTN_CAUSAL_TOP_LEFT && causal != ATTN_CAUSAL_BOTTOM_RIGHT)
     return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_FP16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   const long long bh = static_cast<long long>(B) * H;
   // Grid x and TMA coordinates are 32-bit; grid y is 16-bit.
   if (bh > 0x7fffffffLL || tiles(Nq) > 65535 || tiles(Nk) > 65535) return ATTN_ERR_UNSUPPORTED;
@@ -117,7 +117,7 @@ attn_status check_varlen(int B, int H, int total_q, int total_k, int max_q, int 
   if (causal != ATTN_CAUSAL_NONE && causal != ATTN_CAUSAL_TOP_LEFT && causal != ATTN_CAUSAL_BOTTOM_RIGHT)
     return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_FP16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   const long long bh = static_cast<long long>(B) * H;
   if (bh > 0x7fffffffLL || tiles(max_q) > 65535 || tiles(max_k) > 65535) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(H) * total_q > (1LL << 40) || static_cast<long long>(H) * total_k > (1LL << 40))
@@ -238,6 +238,9 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
   if (d == 64)
     return bf16 ? dispatch_fwd_causal<64, true>(causal, mq, mk, mv, o, lse, pb, sl2, st)
                 : dispatch_fwd_causal<64, false>(causal, mq, mk, mv, o, lse, pb, sl2, st);
+  if (d == 256)
+    return bf16 ? dispatch_fwd_causal<256, true>(causal, mq, mk, mv, o, lse, pb, sl2, st)
+                : dispatch_fwd_causal<256, false>(causal, mq, mk, mv, o, lse, pb, sl2, st);
   return bf16 ? dispatch_fwd_causal<128, true>(causal, mq, mk, mv, o, lse, pb, sl2, st)
               : dispatch_fwd_causal<128, false>(causal, mq, mk, mv, o, lse, pb, sl2, st);
 }
@@ -258,6 +261,7 @@ attn_status dispatch_bwd_causal(int causal, bool det, const CUtensorMap& mq, con
 attn_status bwd_launch(const void* q, const void* k, const void* v, const void* o, const float* lse,
                        const void* dout, void* dq, void* dk, void* dv, void* workspace, const Problem& pb, int d,
                        float scale, int causal, attn_dtype dtype, int phase, bool det, void* stream) {
+  if (d == 256) return ATTN_ERR_UNSUPPORTED;  // see include/attn.h
   const bool bf16 = dtype == ATTN_BF16;
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, q, pb.slabs, pb.rows_q, d, bf16) || !make_map(&mk, k, pb.slabs, pb.rows_k, d, bf16) ||
@@ -404,6 +408,7 @@ attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const v
                             void* stream) {
   const attn_status cs = check_varlen(B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
+  if (d == 256) return ATTN_ERR_UNSUPPORTED;  // forward only
   if (B == 0 || H == 0) return ATTN_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (total_q == 0 || max_seqlen_q == 0) {  // no query rows: dK = dV = 0
@@ -463,6 +468,7 @@ attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
   if (phase < ATTN_BWD_ALL || phase > ATTN_BWD_CONVERT) return ATTN_ERR_INVALID_ARG;
   const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
+  if (d == 256) return ATTN_ERR_UNSUPPORTED;  // forward only
   if (B == 0 || H == 0) return ATTN_OK;
   if (Nk == 0) return Nq == 0 ? ATTN_OK : ATTN_ERR_INVALID_ARG;
   cudaStream_t st0 = static_cast<cudaStream_t>(stream);

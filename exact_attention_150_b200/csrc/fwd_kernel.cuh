@@ -50,7 +50,8 @@ struct FwdLayout {
   static constexpr int kChunks = D / 64;            // 128-byte column chunks per row (>= 1)
   static constexpr int kChunkBytes = kTile * 128;   // one 128-row chunk
   static constexpr int kTileBytes = kTile * D * 2;  // one 128 x D 16-bit tile
-  static constexpr int kSlots = D == 128 ? 5 : 10;  // K/V ring slots
+  static constexpr bool kWide = D == 256;           // see below
+  static constexpr int kSlots = kWide ? 2 : (D == 128 ? 5 : 10);  // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kTileBytes;
   // Exchange between the two softmax warpgroups: row maxima
@@ -69,11 +70,15 @@ struct FwdLayout {
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024 <= 232448 ? kBytes + 1024 : 232448;
   static_assert(kBytes <= 232448, "shared memory budget");
-  // Tensor-memory columns.
+  // Tensor-memory columns.  d = 256: the two S buffers and O take all 512
+  // columns, so Q stays in shared memory (S = Q K^T reads both operands
+  // from there) and the row sums of the 16-bit P are added up by the softmax
+  // threads instead of a row-sum MMA.
   static constexpr uint32_t kColQ = 0;
-  static constexpr uint32_t kColS = 64;    // buffer b at kColS + 128 b
-  static constexpr uint32_t kColO = 320;
-  static constexpr uint32_t kColL = kColO + D;  // 16 columns: row sums of the 16-bit P
+  static constexpr uint32_t kColS = kWide ? 0 : 64;    // buffer b at kColS + 128 b
+  static constexpr uint32_t kColO = kWide ? 256 : 320;
+  static constexpr uint32_t kColL = kColO + D;  // 16 columns: row sums of the 16-bit P (d <= 128)
+  static_assert(kWide ? kColO + D <= 512 : kColL + 16 <= 512, "tensor memory budget");
 };
 
 template <int D, bool BF16, bool CAUSAL>
@@ -241,12 +246,16 @@ __global__ void __launch_bounds__(384, 1)
     };
     // S = Q K^T: A = Q in TMEM (8 columns per K step of 16), B = K K-major
     // (a K step is 32 bytes inside a 128-byte swizzle row).
+    const uint64_t qd = sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
     auto issue_s = [&](int b, uint32_t k_addr) {
       const uint64_t kd = sdesc_sw128(k_addr, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t step = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-        mma_ts(tmem + L::kColS + 128 * b, tmem + L::kColQ + 8 * ks, kd + (step >> 4), kIdS, ks > 0 ? 1u : 0u);
+        if constexpr (L::kWide)  // A = Q in shared memory
+          mma_ss(tmem + L::kColS + 128 * b, qd + (step >> 4), kd + (step >> 4), kIdS, ks > 0 ? 1u : 0u);
+        else
+          mma_ts(tmem + L::kColS + 128 * b, tmem + L::kColQ + 8 * ks, kd + (step >> 4), kIdS, ks > 0 ? 1u : 0u);
       }
     };
     // O += P V: P in the buffer's TMEM columns (key step ks of 16 keys sits
@@ -260,10 +269,12 @@ __global__ void __launch_bounds__(384, 1)
       for (int ks = 0; ks < kTile / 16; ++ks)
         mma_ts(tmem + L::kColO, tmem + L::kColS + 128 * b + 64 * (ks >> 2) + 8 * (ks & 3), vd + 128 * ks, kIdPV,
                (acc || ks > 0) ? 1u : 0u);
+      if constexpr (!L::kWide) {
 #pragma unroll
-      for (int ks = 0; ks < kTile / 16; ++ks)
-        mma_ts(tmem + L::kColL, tmem + L::kColS + 128 * b + 64 * (ks >> 2) + 8 * (ks & 3), ones_d + 32 * ks, kIdL,
-               (acc || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < kTile / 16; ++ks)
+          mma_ts(tmem + L::kColL, tmem + L::kColS + 128 * b + 64 * (ks >> 2) + 8 * (ks & 3), ones_d + 32 * ks, kIdL,
+                 (acc || ks > 0) ? 1u : 0u);
+      }
     };
 
     bool ok = wait_all(q_tmem, 0);
@@ -319,23 +330,25 @@ __global__ void __launch_bounds__(384, 1)
     // Q -> TMEM: this thread copies its row's half of the head dimension
     // (16-byte units of the 128-byte swizzled tile) as 16-bit pairs.
     bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag));
-    if (ok) {
-      constexpr int kUnits = D / 16;  // 16-byte units in half a row
-      const uint8_t* qrow = smem + L::kQOff + (D == 128 ? h * L::kChunkBytes : 0) + row * 128;
-      uint32_t qv[4 * kUnits];
+    if constexpr (!L::kWide) {  // d = 256: Q stays in shared memory
+      if (ok) {
+        constexpr int kUnits = D / 16;  // 16-byte units in half a row
+        const uint8_t* qrow = smem + L::kQOff + (D == 128 ? h * L::kChunkBytes : 0) + row * 128;
+        uint32_t qv[4 * kUnits];
 #pragma unroll
-      for (int u = 0; u < kUnits; ++u) {
-        const int unit = (D == 128 ? u : kUnits * h + u) ^ (row & 7);
-        const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + unit * 16);
-        qv[4 * u] = v4.x; qv[4 * u + 1] = v4.y; qv[4 * u + 2] = v4.z; qv[4 * u + 3] = v4.w;
+        for (int u = 0; u < kUnits; ++u) {
+          const int unit = (D == 128 ? u : kUnits * h + u) ^ (row & 7);
+          const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + unit * 16);
+          qv[4 * u] = v4.x; qv[4 * u + 1] = v4.y; qv[4 * u + 2] = v4.z; qv[4 * u + 3] = v4.w;
+        }
+        if constexpr (D == 128) {
+          tmem_st32(t_row + L::kColQ + 32 * h, qv);
+        } else {
+          tmem_st16(t_row + L::kColQ + 16 * h, qv);
+        }
+        tmem_st_wait();
+        tc_fence_before();
       }
-      if constexpr (D == 128) {
-        tmem_st32(t_row + L::kColQ + 32 * h, qv);
-      } else {
-        tmem_st16(t_row + L::kColQ + 16 * h, qv);
-      }
-      tmem_st_wait();
-      tc_fence_before();
     }
     mbar_arrive(q_tmem);
 
@@ -343,6 +356,7 @@ __global__ void __launch_bounds__(384, 1)
     const float cx = pos_scale ? scale_log2 : 1.f;
     float m_run = -INFINITY;  // running row max (log2 units; stale by < 8)
     float l_run = 0.f;        // this warpgroup's part of sum exp2(score - m_run)
+    float lr_run = 0.f;       // d = 256: the same sum of the 16-bit rounded values
     for (int j = 0; ok && j < n; ++j) {
       const int b = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag));
@@ -384,10 +398,11 @@ __global__ void __launch_bounds__(384, 1)
       // the FMA-pipe exponential, since MUFU throughput bounds them otherwise.
       // A row that has seen no key yet (m_run = -inf; causal with off < 0)
       // uses 0: its scores are all -inf, so p = 0 rather than NaN.
-      float2 su[4];
+      // (d = 256: the rounded ones are summed here too, in sr.)
+      float2 su[4], sr[4];
 #define ATTN_EXP_STORE()                                                                            \
   {                                                                                                 \
-    _Pragma("unroll") for (int i = 0; i < 4; ++i) su[i] = make_float2(0.f, 0.f);                    \
+    _Pragma("unroll") for (int i = 0; i < 4; ++i) su[i] = sr[i] = make_float2(0.f, 0.f);            \
     const float m_use = m_run == -INFINITY ? 0.f : m_run;                                           \
     const float2 cx2 = make_float2(cx, cx), negm2 = make_float2(-m_use, -m_use);                    \
     _Pragma("unroll") for (int c = 0; c < 2; ++c) {                                                 \
@@ -397,6 +412,7 @@ __global__ void __launch_bounds__(384, 1)
         const float2 p = ((i & 3) == 3) ? exp2_poly2(a) : make_float2(ex2(a.x), ex2(a.y));          \
         pk[i] = pack2<BF16>(p.x, p.y);                                                              \
         su[i & 3] = add2(su[i & 3], p);                                                             \
+        if constexpr (L::kWide) sr[i & 3] = add2(sr[i & 3], unpack2<BF16>(pk[i]));                  \
       }                                                                                             \
       tmem_st16(s_col + 16 * c, pk);                                                                \
     }                                                                                               \
@@ -436,9 +452,12 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
           tmem_st32(t_row + L::kColO + (D / 2) * h + 32 * c, r);
         }
-        if (h == 0) tmem_st1(t_row + L::kColL, __float_as_uint(__uint_as_float(tmem_ld1(t_row + L::kColL)) * alpha));
+        if constexpr (!L::kWide) {
+          if (h == 0) tmem_st1(t_row + L::kColL, __float_as_uint(__uint_as_float(tmem_ld1(t_row + L::kColL)) * alpha));
+        }
         if (need) {
           l_run *= alpha;
+          lr_run *= alpha;
           m_run = m_new;
         }
       }
@@ -451,6 +470,10 @@ __global__ void __launch_bounds__(384, 1)
 #undef ATTN_EXP_STORE
       const float2 su01 = add2(su[0], su[1]), su23 = add2(su[2], su[3]);
       l_run += (su01.x + su01.y) + (su23.x + su23.y);
+      if constexpr (L::kWide) {
+        const float2 sr01 = add2(sr[0], sr[1]), sr23 = add2(sr[2], sr[3]);
+        lr_run += (sr01.x + sr01.y) + (sr23.x + sr23.y);
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
@@ -458,6 +481,7 @@ __global__ void __launch_bounds__(384, 1)
     // Epilogue: combine the two warpgroups' row sums, then each warpgroup
     // writes its half of the head dimension of O.
     xsum[h * kTile + row] = l_run;
+    if constexpr (L::kWide) xsum[(2 + h) * kTile + row] = lr_run;
     mbar_arrive(xsum_bar);
     if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(xsum_bar, 0, abort_flag));
     if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort_flag));
@@ -469,7 +493,11 @@ __global__ void __launch_bounds__(384, 1)
       // ~2^-126 rather than 0 for a masked score.)
       // (tcgen05.ld is warp-collective: every lane loads, then selects.)
       const bool empty = m_run == -INFINITY;
-      const float l_tc = __uint_as_float(tmem_ld1(t_row + L::kColL));
+      float l_tc;
+      if constexpr (L::kWide)
+        l_tc = lr_run + xsum[(2 + (h ^ 1)) * kTile + row];
+      else
+        l_tc = __uint_as_float(tmem_ld1(t_row + L::kColL));
       const float inv = empty ? 0.f : 1.f / l_tc;
       const bool live = qt * kTile + row < nq;  // padding rows of a ragged tile are not stored
       const size_t grow = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile + row;

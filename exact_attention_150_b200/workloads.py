@@ -65,8 +65,10 @@ SWEEP = {n: Workload(f"sweep{n}", 4, 32, n, 128, "fp16", False, False, 1003)
          for n in (512, 1024, 2048, 4096, 8192)}
 TRAIN_D64 = Workload("train_d64", 2, 16, 4096, 64, "fp16", True, True, 1004)
 LONG_CTX = Workload("long_ctx", 1, 16, 16384, 128, "bf16", True, True, 1005, 0.5)
+# Head dimension 256 (forward only): the long-context shape at d = 256.
+FWD_D256 = Workload("fwd_d256", 1, 16, 16384, 256, "bf16", True, False, 1006, 0.5)
 
-ALL = [TINY, LAYER_7B, *SWEEP.values(), TRAIN_D64, LONG_CTX]
+ALL = [TINY, LAYER_7B, *SWEEP.values(), TRAIN_D64, LONG_CTX, FWD_D256]
 
 
 def by_name(name: str) -> Workload:

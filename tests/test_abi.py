@@ -99,7 +99,7 @@ def test_no_keys_is_invalid(lib):
     assert _bwd(Nk=0, Nq=0) == native.ATTN_OK
 
 
-@pytest.mark.parametrize("kw", [dict(d=96), dict(d=256), dict(d=32), dict(d=0), dict(dtype=2), dict(dtype=-1),
+@pytest.mark.parametrize("kw", [dict(d=96), dict(d=512), dict(d=32), dict(d=0), dict(dtype=2), dict(dtype=-1),
                                 dict(Nq=65535 * 128 + 1), dict(Nk=65535 * 128 + 1)])
 def test_unsupported_shapes(lib, kw):
     assert _fwd(**kw) == native.ATTN_ERR_UNSUPPORTED
@@ -237,3 +237,15 @@ def test_selftest_rejects_bad_limits(lib, limit_us):
 
 def test_selftest_rejects_null_result(lib):
     assert native.load().attn_selftest_wait_timeout(1000, None, None) == native.ATTN_ERR_INVALID_ARG
+
+
+def test_head_dim_256_is_forward_only(lib):
+    """d = 256 passes the forward's checks (not called here: the pointers are
+    fake) and is refused by every backward entry point before any work."""
+    assert _bwd(d=256) == native.ATTN_ERR_UNSUPPORTED
+    assert _bwd(d=256, Nq=0, dq=None, dout=None, q=None, o=None, lse=None) == native.ATTN_ERR_UNSUPPORTED
+    assert _bwd_varlen(d=256) == native.ATTN_ERR_UNSUPPORTED
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, workspace=FAKE,
+                B=1, H=1, Nq=128, Nk=128, d=256, scale=0.1, causal=0, dtype=native.ATTN_BF16, stream=None)
+    assert native.attn_bwd_deterministic(**args) == native.ATTN_ERR_UNSUPPORTED
+    assert _fwd(d=256, q=None) == native.ATTN_ERR_INVALID_ARG  # validated like any supported d

@@ -141,6 +141,48 @@ def test_forward_bottom_right_single_query_is_noncausal():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("causal", [False, True, "bottom_right"])
+@pytest.mark.parametrize("nq,nk", [(128, 128), (300, 300), (640, 640), (100, 700), (500, 130)])
+def test_forward_head_dim_256(dtype, causal, nq, nk):
+    """d = 256: Q stays in shared memory, the rounded-P row sums come from
+    the softmax threads, and the K/V ring has two slots."""
+    q, k, v = draw(1, 2, nq, nk, 256, dtype, seed=41 + nq + nk)
+    check_all_slices(q, k, v, causal, 1.0 / math.sqrt(256), f"d256 Nq{nq} Nk{nk} {dtype} causal={causal}")
+
+
+def test_forward_head_dim_256_varlen():
+    lens = [130, 1, 400, 0, 255]
+    H, d = 2, 256
+    qs, ks, vs = [], [], []
+    for b, n in enumerate(lens):
+        q, k, v = draw(1, H, n, n, d, torch.bfloat16, seed=51 + b)
+        qs.append(q[0]); ks.append(k[0]); vs.append(v[0])
+    q, k, v = (torch.cat(t, dim=1).contiguous() for t in (qs, ks, vs))
+    cu = torch.tensor([0] + torch.tensor(lens).cumsum(0).tolist(), dtype=torch.int32)
+    o, lse = native.forward_varlen(*(t.to(DEV) for t in (q, k, v)), cu.to(DEV), cu.to(DEV), max(lens), max(lens),
+                                   causal=True)
+    torch.cuda.synchronize()
+    native.device_status()
+    o, lse = o.cpu(), lse.cpu()
+    for b in range(len(lens)):
+        a, z = int(cu[b]), int(cu[b + 1])
+        if z == a:
+            continue
+        for h in range(H):
+            ro, rl, _ = oracle.forward(parity.f64(q[h, a:z]), parity.f64(k[h, a:z]), parity.f64(v[h, a:z]),
+                                       1 / math.sqrt(d), True)
+            parity.assert_o(parity.f64(o[h, a:z]), ro, torch.bfloat16, f"d256 varlen seq {b} head {h}")
+            parity.assert_lse(parity.f64(lse[h, a:z]), rl, f"d256 varlen seq {b} head {h}")
+
+
+def test_backward_head_dim_256_raises():
+    q = torch.zeros(1, 1, 128, 256, dtype=torch.bfloat16, device=DEV)
+    lse = torch.zeros(1, 1, 128, device=DEV)
+    with pytest.raises(native.AttnError, match="status 2"):
+        native.backward(q, q, q, q, lse, q)
+
+
 def test_forward_empty_problems():
     for shape_q, shape_k in (((0, 2, 128, 64), (0, 2, 128, 64)), ((1, 2, 0, 64), (1, 2, 64, 64))):
         q = torch.zeros(shape_q, dtype=torch.bfloat16, device=DEV)
