@@ -35,7 +35,9 @@
  *   rows i < Nq - Nk) has an empty softmax: O = 0, LSE = -inf, dQ = 0.
  * LSE.  lse[b][h][i] = ln sum_j exp(scale * q_i . k_j) over the unmasked j:
  *   the natural-log row log-sum-exp of the scaled scores, in fp32.
- * Supported shapes.  d in {64, 128}; any Nq, Nk >= 0 (the kernels work in
+ * Supported shapes.  d in {64, 128}, and 256 for the forward calls only
+ *   (every backward entry point returns ATTN_ERR_UNSUPPORTED for d = 256:
+ *   its dV and dK accumulators alone would fill tensor memory); any Nq, Nk >= 0 (the kernels work in
  *   tiles of 128 rows and mask a ragged last tile); causal with any Nq, Nk.
  *   The tile counts ceil(Nq / 128) and ceil(Nk / 128) must not exceed 65535
  *   and B*H must fit in an int; other shapes return ATTN_ERR_UNSUPPORTED.
