@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload long_ctx] [--seq N] [--no-cpu-baseline] [--e2e-steps E]
+                    [--deterministic] [--varlen]
 
 One step is one pass of the whole hot path over one batch of synthetic input:
 the forward kernel, then the three backward kernels (D preprocess, main,
@@ -15,6 +16,9 @@ Rank 0 prints ONE JSON line.  For N > 1 (torchrun, one process per GPU) every
 rank runs an independent replica of the workload: the path has no exchange
 step, so there is no collective on the data path; the timing is the max over
 ranks (an all-reduce of the elapsed time only).
+
+--varlen times a packed variable-length batch instead (attn_fwd_varlen and
+attn_bwd_varlen on a seeded length mix; see workloads.VARLEN_MIX).
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on a
 bounded sample of the same workload on the host cores, and prints the same
@@ -56,6 +60,7 @@ def parse_args(argv=None):
     p.add_argument("--seq", type=int, default=None, help="override the sequence length (profiling runs)")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--varlen", action="store_true", help="time a packed variable-length batch")
     p.add_argument("--deterministic", action="store_true",
                    help="time the bit-reproducible backward (attn_bwd_deterministic) instead of attn_bwd")
     return p.parse_args(argv)
@@ -407,10 +412,104 @@ def run_ours(args):
     return 0
 
 
+def run_varlen(args):
+    """The packed variable-length batch: forward then backward per step."""
+    import torch
+    rank, world, local_rank = dist_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(device)
+    from exact_attention_150_b200 import native, workloads
+    native.load()
+    m = workloads.VARLEN_MIX
+    lens = workloads.varlen_lengths(m["seed"], m["total"], m["lo"], m["hi"])
+    H, d = m["H"], m["d"]
+    dtype = torch.bfloat16 if m["dtype"] == "bf16" else torch.float16
+    q, k, v, do, cu = (t.to(device) for t in workloads.make_varlen_inputs(lens, H, d, dtype, m["seed"],
+                                                                           m["input_scale"]))
+    mx = max(lens)
+    scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty(H, q.shape[1], dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(native.attn_bwd_varlen_workspace_bytes(len(lens), H, q.shape[1], mx, d), dtype=torch.uint8,
+                     device=device)
+    stream = torch.cuda.current_stream(device)
+    fwd_flops = sum(4.0 * H * n * n * d / (2 if m["causal"] else 1) for n in lens)
+    bwd_flops = 2.5 * fwd_flops
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        native.forward_varlen(q, k, v, cu, cu, mx, mx, causal=m["causal"], scale=scale, out=o, lse=lse)
+        if ev is not None:
+            ev[1].record(stream)
+        native.backward_varlen(q, k, v, o, lse, do, cu, cu, mx, mx, causal=m["causal"], scale=scale, dq=dq, dk=dk,
+                               dv=dv, workspace=ws, deterministic=args.deterministic)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize(device)
+    native.device_status()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    native.device_status()
+    max_ms = max_over_ranks(start.elapsed_time(end), world, device)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    peaks, peak_src = load_peaks()
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    bwd_tf = bwd_flops / bwd_ms / 1e9
+    line = {
+        "metric": METRIC, "value": aggregate(fwd_flops + bwd_flops, args.steps, world, max_ms), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": m["dtype"],
+        "data": "synthetic: seeded i.i.d. N(0,1) packed Q, K, V, dO (x%g)" % m["input_scale"],
+        "config": {"workload": f"{m['name']}: packed causal {m['dtype']} H{H} d{d}, {len(lens)} sequences, "
+                               f"{sum(lens)} tokens, lengths {min(lens)}..{max(lens)}",
+                   "lengths": lens, "backward": "deterministic" if args.deterministic else "atomic dQ",
+                   "l2": "no flush: packed Q, K, V, dO of %d MB each" % (H * sum(lens) * d * 2 // 2**20),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "fwd_tflops": fwd_flops / fwd_ms / 1e9, "bwd_tflops": bwd_tf,
+        "kernels": {"fwd_kernel (varlen)": {"ms": fwd_ms, "tflops": fwd_flops / fwd_ms / 1e9},
+                    "bwd (varlen, all kernels)": {"ms": bwd_ms, "tflops": bwd_tf}},
+        "roofline": {"kernel": "bwd (varlen, all kernels)", "bound": "tensor", "achieved": bwd_tf, "peak": peak_sus,
+                     "unit": "TFLOP/s", "frac": bwd_tf / peak_sus, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained"},
+        "clocks": clocks.summary(), "e2e": None, "gpu_launches": 4 * args.steps,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.varlen:
+        return run_varlen(args)
     return run_ours(args)
 
 

@@ -99,3 +99,37 @@ def draw(B, H, Nq, Nk, d, dtype, seed, input_scale=1.0, with_grad=False, device=
             t.mul_(input_scale)
         out.append(t.to(dtype).to(device))
     return tuple(out)
+
+
+# Packed variable-length batch: a seeded mix of causal self-attention
+# sequences (lengths uniform in [1024, 16384], the last one cut so that the
+# batch holds 65536 tokens), H = 16, d = 128, bf16, inputs scaled by 0.5.
+VARLEN_MIX = dict(name="varlen_mix", H=16, d=128, dtype="bf16", causal=True, seed=1007, total=65536, lo=1024,
+                  hi=16384, input_scale=0.5)
+
+
+def varlen_lengths(seed: int, total: int, lo: int, hi: int) -> list[int]:
+    """Seeded sequence lengths, uniform in [lo, hi], summing to total."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    lens: list[int] = []
+    while sum(lens) < total:
+        n = int(torch.randint(lo, hi + 1, (1,), generator=g))
+        lens.append(min(n, total - sum(lens)))
+    return lens
+
+
+def make_varlen_inputs(lengths, H: int, d: int, dtype: torch.dtype, seed: int, input_scale: float = 1.0):
+    """Packed head-major Q, K, V, dO [H, total, d] (self-attention: every
+    sequence has as many keys as queries) and the int32 offsets [B + 1]."""
+    total = sum(lengths)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    out = []
+    for _ in range(4):
+        t = torch.randn((H, total, d), generator=g, dtype=torch.float32)
+        if input_scale != 1.0:
+            t.mul_(input_scale)
+        out.append(t.to(dtype))
+    cu = torch.tensor([0] + torch.tensor(lengths).cumsum(0).tolist(), dtype=torch.int32)
+    return (*out, cu)
