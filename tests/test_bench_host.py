@@ -77,3 +77,17 @@ def test_reference_arm_other_ranks_exit_quietly():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--seq", "256",
                           "--steps", "1", "--warmup", "0"], capture_output=True, text=True, env=env, timeout=300)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_varlen_mix_is_seeded_and_bounded():
+    import torch
+    from exact_attention_150_b200 import workloads
+    m = workloads.VARLEN_MIX
+    a = workloads.varlen_lengths(m["seed"], m["total"], m["lo"], m["hi"])
+    b = workloads.varlen_lengths(m["seed"], m["total"], m["lo"], m["hi"])
+    assert a == b and sum(a) == m["total"]
+    assert all(1 <= n <= m["hi"] for n in a) and all(n >= m["lo"] for n in a[:-1])
+    q, k, v, do, cu = workloads.make_varlen_inputs([3, 5], 2, 8, torch.bfloat16, 7)
+    assert q.shape == (2, 8, 8) and cu.tolist() == [0, 3, 8] and cu.dtype == torch.int32
+    q2 = workloads.make_varlen_inputs([3, 5], 2, 8, torch.bfloat16, 7)[0]
+    assert torch.equal(q, q2)
