@@ -151,6 +151,12 @@ def test_forward_head_dim_256(dtype, causal, nq, nk):
     check_all_slices(q, k, v, causal, 1.0 / math.sqrt(256), f"d256 Nq{nq} Nk{nk} {dtype} causal={causal}")
 
 
+@pytest.mark.parametrize("scale", [0.0, -0.05])
+def test_forward_head_dim_256_other_scales(scale):
+    q, k, v = draw(1, 2, 300, 300, 256, torch.bfloat16, seed=47)
+    check_all_slices(q, k, v, True, scale, f"d256 scale {scale}")
+
+
 def test_forward_head_dim_256_varlen():
     lens = [130, 1, 400, 0, 255]
     H, d = 2, 256
