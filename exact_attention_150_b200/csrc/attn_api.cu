@@ -32,10 +32,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3D view [B*H][N][d] of a contiguous 16-bit tensor, read in boxes of 64
-// columns (128 bytes) x 128 rows of one (b, h) slice with the 128-byte
-// swizzle the MMA descriptors expect.  Rows past N read as zeros, so a
-// ragged last tile never touches the next slice.
+// 3D view [slabs][N][d] of a contiguous 16-bit tensor (a slab is one
+// (batch, head) slice of a dense batch, or one head of a packed
+// variable-length batch), read in boxes of 64 columns (128 bytes) x 128 rows
+// of one slab with the 128-byte swizzle the MMA descriptors expect.  Rows
+// past N read as zeros, so a ragged last tile never touches the next slab.
 bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;

@@ -5,7 +5,9 @@
 // 核心原理", part 2 item 3).  Three kernels:
 //
 //   bwd_pre_kernel    D_i = sum_c dO_ic O_ic, -log2(e) * LSE_i, and dQacc = 0
-//   bwd_main_kernel   one CTA per (key tile j, batch*head): K_j, V_j stay in
+//   bwd_main_kernel   one CTA per (key tile j, problem), a problem being one
+//                     (batch, head) slice or one sequence of one head of a
+//                     packed variable-length batch: K_j, V_j stay in
 //                     shared memory; for every query tile i that sees them
 //                       S'^T  = K_j Q_i^T - LSE_i / scale   (tcgen05, TMEM)
 //                       dP'^T = V_j dO_i^T - D_i            (tcgen05, TMEM)
