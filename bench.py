@@ -321,7 +321,9 @@ def run_ours(args):
     value = aggregate(step_flops, args.steps, world, max_ms)
     peaks, peak_src = load_peaks()
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    kernels = {"fwd_kernel": {"ms": fwd_ms, "tflops": w.fwd_flops() / fwd_ms / 1e9}}
+    # Forward algorithmic bytes: read Q, K, V, write O (16-bit) and LSE (fp32).
+    fwd_bytes = w.B * w.H * (2 * (2 * w.N + 2 * w.N) * w.d + 4 * w.N)
+    kernels = {"fwd_kernel": {"ms": fwd_ms, "tflops": w.fwd_flops() / fwd_ms / 1e9, "gbs": fwd_bytes / fwd_ms / 1e6}}
     if w.backward and args.deterministic:
         det_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
         kernels["bwd_deterministic (order counters + 3 kernels)"] = {"ms": det_ms,
