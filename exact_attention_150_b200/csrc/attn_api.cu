@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "attn.h"
 #include "bwd_kernel.cuh"
@@ -78,9 +80,27 @@ attn_status check_common(int B, int H, int Nq, int Nk, int d, int causal, attn_d
   return ATTN_OK;
 }
 
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device):
+// the attribute persists, and setting it on every launch costs host time
+// that small problems notice.
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  const cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess) return ge;
+  const std::pair<const void*, int> key(reinterpret_cast<const void*>(kernel), dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count(key)) return cudaSuccess;
+  }
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) {
+    std::lock_guard<std::mutex> lock(mu);
+    done.insert(key);
+  }
+  return e;
 }
 
 // A launch's problems.  Dense batches: one tensor-map slab per (batch,
