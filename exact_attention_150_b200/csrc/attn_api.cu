@@ -74,8 +74,10 @@ attn_status check_common(int B, int H, int Nq, int Nk, int d, int causal, attn_d
   if (dtype != ATTN_FP16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
   if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   const long long bh = static_cast<long long>(B) * H;
-  // Grid x and TMA coordinates are 32-bit; grid y is 16-bit.
+  // TMA coordinates are 32-bit, and so is the one-dimensional grid of
+  // (problem, tile) CTAs.
   if (bh > 0x7fffffffLL || tiles(Nq) > 65535 || tiles(Nk) > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (bh * tiles(Nq) > 0x7fffffffLL || bh * tiles(Nk) > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if (bh * Nq > (1LL << 40) || bh * Nk > (1LL << 40)) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
@@ -110,14 +112,19 @@ cudaError_t set_smem(K kernel, int bytes) {
 struct Problem {
   int slabs;               // slab count of the tensor maps
   int rows_q, rows_k;      // rows per slab
-  int problems;            // grid x: B*H
-  int qtiles, ktiles;      // grid y: tiles of the longest query / key sequence
+  int problems;            // B*H
+  int qtiles, ktiles;      // tiles of the longest query / key sequence
   const int* cu_q = nullptr;
   const int* cu_k = nullptr;
   int H = 1;
   int bottom_right = 0;
   bool packed = false;     // variable-length batch
 };
+
+// Average rows per problem of a tensor with rows_per_slab rows in each slab.
+double avg_rows(int rows_per_slab, const Problem& pb) {
+  return pb.problems > 0 ? static_cast<double>(rows_per_slab) * pb.slabs / pb.problems : 0.0;
+}
 
 Problem dense_problem(int B, int H, int Nq, int Nk, int causal) {
   Problem p;
@@ -141,6 +148,7 @@ attn_status check_varlen(int B, int H, int total_q, int total_k, int max_q, int 
   if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   const long long bh = static_cast<long long>(B) * H;
   if (bh > 0x7fffffffLL || tiles(max_q) > 65535 || tiles(max_k) > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (bh * tiles(max_q) > 0x7fffffffLL || bh * tiles(max_k) > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(H) * total_q > (1LL << 40) || static_cast<long long>(H) * total_k > (1LL << 40))
     return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
@@ -191,9 +199,11 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   using L = attn::FwdLayout<D>;
   auto kern = attn::fwd_kernel<D, BF16, CAUSAL>;
   if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
-  dim3 grid(pb.problems, pb.qtiles);
+  // Every CTA of a problem streams its K and V.
+  const int group = attn::order_group(4.0 * D * avg_rows(pb.rows_k, pb), pb.problems);
+  const unsigned grid = static_cast<unsigned>(pb.problems) * static_cast<unsigned>(pb.qtiles);
   kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, pb.cu_q, pb.cu_k, pb.H, pb.rows_q,
-                                     pb.rows_k, pb.bottom_right, scale_log2);
+                                     pb.rows_k, pb.bottom_right, scale_log2, pb.problems, pb.qtiles, group);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -221,10 +231,18 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_MAIN) {
     auto kern = attn::bwd_main_kernel<D, BF16, CAUSAL, DET>;
     if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
-    dim3 grid(pb.problems, pb.ktiles);
+    // Every CTA of a problem streams its Q and dO rows, their LSE and D, and
+    // adds into its dQ accumulator rows.  The deterministic mode keeps
+    // problem-fastest order: its key tiles take turns on each query tile, and
+    // a problem whose key tiles were all resident at once would leave key
+    // tile j waiting about 2j steps.
+    const int group =
+        DET ? pb.problems : attn::order_group((8.0 * D + 8.0) * avg_rows(pb.rows_q, pb), pb.problems);
+    const unsigned grid = static_cast<unsigned>(pb.problems) * static_cast<unsigned>(pb.ktiles);
     kern<<<grid, 512, L::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, dqacc, static_cast<uint16_t*>(dk),
                                        static_cast<uint16_t*>(dv), dq_order, pb.cu_q, pb.cu_k, pb.H, pb.rows_q,
-                                       pb.rows_k, pb.bottom_right, pb.qtiles, scale, scale * 1.4426950408889634f);
+                                       pb.rows_k, pb.bottom_right, pb.qtiles, scale, scale * 1.4426950408889634f,
+                                       pb.problems, pb.ktiles, group);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_CONVERT) {

@@ -53,6 +53,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "tile_order.h"
 
 namespace attn {
 
@@ -170,7 +171,8 @@ __global__ void __launch_bounds__(512, 1)
                     const float* __restrict__ dvec, const float* __restrict__ nlse2, float* __restrict__ dqacc,
                     uint16_t* __restrict__ dk_ptr, uint16_t* __restrict__ dv_ptr, int* __restrict__ dq_order,
                     const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H, int Nq, int Nk,
-                    int bottom_right, int order_stride, float scale, float scale_log2) {
+                    int bottom_right, int order_stride, float scale, float scale_log2, int problems,
+                    int grid_tiles, int group) {
   using L = BwdLayout<D>;
   constexpr bool kDqT = (D == 128);  // dQ formed transposed (see above)
   constexpr uint32_t kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 256 + D;
@@ -200,10 +202,14 @@ __global__ void __launch_bounds__(512, 1)
   // and rows [q0, q0 + nq) / [k0, k0 + nk) of it (one slab per (batch,
   // head) for dense batches; one per head for packed variable-length
   // batches, sequence b's rows from the offsets clamped to the slab).
-  int z = blockIdx.x, q0 = 0, k0 = 0, nq = Nq, nk = Nk;
+  // The grid is one-dimensional, in the grouped launch order of
+  // tile_order.h: px is the problem, j the key tile.
+  int px, j;
+  grouped_order(blockIdx.x, problems, grid_tiles, group, &px, &j);
+  int z = px, q0 = 0, k0 = 0, nq = Nq, nk = Nk;
   if (cu_q != nullptr) {
-    const int b = static_cast<int>(blockIdx.x) / H;
-    z = static_cast<int>(blockIdx.x) - b * H;
+    const int b = px / H;
+    z = px - b * H;
     auto clamp = [](int v, int hi) { return v < 0 ? 0 : (v > hi ? hi : v); };
     q0 = clamp(cu_q[b], Nq);
     k0 = clamp(cu_k[b], Nk);
@@ -215,7 +221,7 @@ __global__ void __launch_bounds__(512, 1)
     // also keeps the order counters of the deterministic mode in range.
     nq = nq < order_stride * kBwdTile ? nq : order_stride * kBwdTile;
   }
-  const int j = blockIdx.y;  // key tile; causal: small j has the most work and launches first
+  // Key tile j; causal: small j has the most work and launches first.
   if (j * kBwdTile >= nk) return;  // a sequence shorter than the grid
   const int nqt = (nq + kBwdTile - 1) / kBwdTile;  // the last tiles may be ragged
   // Causal: query q sees key k iff k <= q + off (off = 0 top-left,
@@ -565,7 +571,7 @@ __global__ void __launch_bounds__(512, 1)
       // never decreases with it), so this CTA is contributor number j of
       // every query tile it covers.  It reduces into the tile only after the
       // 4 drain warps of contributors 0..j-1 have each counted theirs.
-      int* turn = DET ? dq_order + static_cast<size_t>(blockIdx.x) * order_stride + (i0 + it) : nullptr;
+      int* turn = DET ? dq_order + static_cast<size_t>(px) * order_stride + (i0 + it) : nullptr;
       auto await_turn = [&]() {
         if constexpr (DET) {
           if (!__all_sync(0xffffffffu, wait_turn(turn, 4 * j, abort_flag))) return false;

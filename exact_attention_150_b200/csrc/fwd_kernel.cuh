@@ -40,6 +40,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "tile_order.h"
 
 namespace attn {
 
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o_ptr,
                float* __restrict__ lse_ptr, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H,
-               int Nq, int Nk, int bottom_right, float scale_log2) {
+               int Nq, int Nk, int bottom_right, float scale_log2, int problems, int grid_tiles, int group) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -116,10 +117,14 @@ __global__ void __launch_bounds__(384, 1)
   // batches have one slab per head and take sequence b's rows from the
   // offsets, clamped to the slab: bad offsets can give wrong values but
   // never address outside the tensors.
-  int z = blockIdx.x, q0 = 0, k0 = 0, nq = Nq, nk = Nk;
+  // The grid is one-dimensional, in the grouped launch order of
+  // tile_order.h: px is the problem, ty the query tile in launch order.
+  int px, ty;
+  grouped_order(blockIdx.x, problems, grid_tiles, group, &px, &ty);
+  int z = px, q0 = 0, k0 = 0, nq = Nq, nk = Nk;
   if (cu_q != nullptr) {
-    const int b = static_cast<int>(blockIdx.x) / H;
-    z = static_cast<int>(blockIdx.x) - b * H;
+    const int b = px / H;
+    z = px - b * H;
     auto clamp = [](int v, int hi) { return v < 0 ? 0 : (v > hi ? hi : v); };
     q0 = clamp(cu_q[b], Nq);
     k0 = clamp(cu_k[b], Nk);
@@ -130,9 +135,9 @@ __global__ void __launch_bounds__(384, 1)
   }
   const int nqt = (nq + kTile - 1) / kTile;  // the last tiles may be ragged
   const int nkt = (nk + kTile - 1) / kTile;
-  if (static_cast<int>(blockIdx.y) >= nqt) return;  // a sequence shorter than the grid
+  if (ty >= nqt) return;  // a sequence shorter than the grid
   // Causal: the heaviest query tiles are launched first.
-  const int qt = CAUSAL ? (nqt - 1 - static_cast<int>(blockIdx.y)) : static_cast<int>(blockIdx.y);
+  const int qt = CAUSAL ? (nqt - 1 - ty) : ty;
   // Key tiles this query tile sees.  Causal: query i sees key k iff
   // k <= i + off (off = 0 top-left, nk - nq bottom-right).
   const int off = bottom_right ? nk - nq : 0;

@@ -39,8 +39,10 @@
  *   (every backward entry point returns ATTN_ERR_UNSUPPORTED for d = 256:
  *   its dV and dK accumulators alone would fill tensor memory); any Nq, Nk >= 0 (the kernels work in
  *   tiles of 128 rows and mask a ragged last tile); causal with any Nq, Nk.
- *   The tile counts ceil(Nq / 128) and ceil(Nk / 128) must not exceed 65535
- *   and B*H must fit in an int; other shapes return ATTN_ERR_UNSUPPORTED.
+ *   The tile counts ceil(Nq / 128) and ceil(Nk / 128) must not exceed 65535,
+ *   and B*H and B*H times each tile count must fit in an int (for the packed
+ *   calls, with the longest sequence's tile counts); other shapes return
+ *   ATTN_ERR_UNSUPPORTED.
  * Empty problems.  B, H, Nq or Nk may be 0.  A call with no query rows
  *   (B*H*Nq == 0) is valid and does nothing, except that attn_bwd then writes
  *   dK = dV = 0 (their rows exist but no query reaches them).  Nq > 0 with

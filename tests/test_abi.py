@@ -100,7 +100,9 @@ def test_no_keys_is_invalid(lib):
 
 
 @pytest.mark.parametrize("kw", [dict(d=96), dict(d=512), dict(d=32), dict(d=0), dict(dtype=2), dict(dtype=-1),
-                                dict(Nq=65535 * 128 + 1), dict(Nk=65535 * 128 + 1)])
+                                dict(Nq=65535 * 128 + 1), dict(Nk=65535 * 128 + 1),
+                                # B*H times the tile count exceeds the one-dimensional grid
+                                dict(B=1 << 16, H=1 << 10, Nq=64 * 128), dict(B=1 << 16, H=1 << 10, Nk=64 * 128)])
 def test_unsupported_shapes(lib, kw):
     assert _fwd(**kw) == native.ATTN_ERR_UNSUPPORTED
     assert _bwd(**kw) == native.ATTN_ERR_UNSUPPORTED
@@ -213,6 +215,8 @@ def test_varlen_validation(lib, fn):
     assert fn(dtype=5) == native.ATTN_ERR_UNSUPPORTED
     assert fn(causal=3) == native.ATTN_ERR_INVALID_ARG
     assert fn(max_q=65535 * 128 + 1) == native.ATTN_ERR_UNSUPPORTED
+    assert fn(B=1 << 16, H=1 << 10, max_q=64 * 128) == native.ATTN_ERR_UNSUPPORTED
+    assert fn(B=1 << 16, H=1 << 10, max_k=64 * 128) == native.ATTN_ERR_UNSUPPORTED
     assert fn(cu_q=None) == native.ATTN_ERR_INVALID_ARG
     assert fn(cu_k=FAKE + 2) == native.ATTN_ERR_INVALID_ARG  # offsets must be 4-byte aligned
     assert fn(q=FAKE + 8) == native.ATTN_ERR_INVALID_ARG
