@@ -242,3 +242,20 @@ def test_sweep_workload_sampled(n):
     for s, ref, lref in zip(slices, refs, lrefs):
         parity.assert_o(parity.f64(of[s][rows]), ref, q.dtype, f"{w.label()} slice {s}")
         parity.assert_lse(parity.f64(lf[s][rows]), lref, f"{w.label()} slice {s}")
+
+
+@pytest.mark.parametrize("n", [4096, 8192])
+def test_causal_sweep_workload_sampled(n):
+    # Causal bf16 on the sweep's batch shape: sampled slices (in different
+    # launch groups) and rows, including both sides of tile boundaries.
+    w = workloads.CAUSAL_SWEEP[n]
+    q, k, v = workloads.make_inputs(w, with_grad=False)
+    o, lse = run_forward(q, k, v, w.causal, w.scale)
+    B, H = w.B, w.H
+    slices = [0, 9, 70, B * H - 1]
+    rows = _sampled_rows(n, 48, n + 1)
+    refs, lrefs = parity.oracle_forward_slices(q, k, v, w.scale, w.causal, slices, rows)
+    of, lf = o.reshape(B * H, n, w.d), lse.reshape(B * H, n)
+    for s, ref, lref in zip(slices, refs, lrefs):
+        parity.assert_o(parity.f64(of[s][rows]), ref, q.dtype, f"{w.label()} slice {s}")
+        parity.assert_lse(parity.f64(lf[s][rows]), lref, f"{w.label()} slice {s}")
