@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -39,14 +40,18 @@ EncodeTiledFn encode_fn() {
 // variable-length batch), read in boxes of 64 columns (128 bytes) x 128 rows
 // of one slab with the 128-byte swizzle the MMA descriptors expect.  Rows
 // past N read as zeros, so a ragged last tile never touches the next slab.
-bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16) {
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16, bool e4m3 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  // Boxes are 128 bytes wide (64 16-bit or 128 8-bit elements) by 128 rows.
+  const cuuint64_t eb = e4m3 ? 1 : 2;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTile), 1};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * eb, static_cast<cuuint64_t>(N) * d * eb};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(kTile), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+  const CUtensorMapDataType type = e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                        : (bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  const CUresult r = fn(map, type, 3,
                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -193,17 +198,18 @@ WsLayout ws_layout(const Problem& pb, int d) {
   return w;
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool F8 = false>
 attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse,
-                       const Problem& pb, float scale_log2, cudaStream_t st) {
-  using L = attn::FwdLayout<D>;
-  auto kern = attn::fwd_kernel<D, BF16, CAUSAL>;
+                       const Problem& pb, float scale_log2, cudaStream_t st, float o_scale = 1.f) {
+  using L = attn::FwdLayout<D, F8>;
+  auto kern = attn::fwd_kernel<D, BF16, CAUSAL, F8>;
   if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
   // Every CTA of a problem streams its K and V.
-  const int group = attn::order_group(4.0 * D * avg_rows(pb.rows_k, pb), pb.problems);
+  const int group = attn::order_group(2.0 * L::kRowBytes * avg_rows(pb.rows_k, pb), pb.problems);
   const unsigned grid = static_cast<unsigned>(pb.problems) * static_cast<unsigned>(pb.qtiles);
   kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, pb.cu_q, pb.cu_k, pb.H, pb.rows_q,
-                                     pb.rows_k, pb.bottom_right, scale_log2, pb.problems, pb.qtiles, group);
+                                     pb.rows_k, pb.bottom_right, scale_log2, pb.problems, pb.qtiles, group,
+                                     o_scale);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -402,6 +408,31 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return ATTN_ERR_INVALID_ARG;
   return fwd_impl(q, k, v, o, lse, dense_problem(B, H, Nq, Nk, causal), d, scale, causal, dtype, stream);
+}
+
+attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                         int Nk, int d, float scale, float descale_q, float descale_k, float descale_v, int causal,
+                         void* stream) {
+  const attn_status cs = check_common(B, H, Nq, Nk, d, causal, ATTN_BF16);
+  if (cs != ATTN_OK) return cs;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!std::isfinite(descale_q) || !std::isfinite(descale_k) || !std::isfinite(descale_v) || !std::isfinite(scale))
+    return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || Nq == 0) return ATTN_OK;  // no query rows: nothing to write
+  if (Nk == 0) return ATTN_ERR_INVALID_ARG;         // a softmax over no keys is undefined
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_INVALID_ARG;
+  const Problem pb = dense_problem(B, H, Nq, Nk, causal);
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, pb.slabs, pb.rows_q, d, true, true) || !make_map(&mk, k, pb.slabs, pb.rows_k, d, true, true) ||
+      !make_map(&mv, v, pb.slabs, pb.rows_k, d, true, true))
+    return ATTN_ERR_CUDA;
+  // The scores are scale * (descale_q q) . (descale_k k): one factor, in log2 units.
+  const float sl2 = scale * descale_q * descale_k * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return causal ? launch_fwd<128, true, true, true>(mq, mk, mv, o, lse, pb, sl2, st, descale_v)
+                : launch_fwd<128, true, false, true>(mq, mk, mv, o, lse, pb, sl2, st, descale_v);
 }
 
 attn_status attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,

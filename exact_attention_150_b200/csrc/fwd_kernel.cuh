@@ -46,13 +46,18 @@ namespace attn {
 
 constexpr int kTile = 128;  // rows of a query tile and of a key/value tile
 
-template <int D>
+// F8: Q, K and V are E4M3 bytes (d = 128 only) instead of 16-bit values.
+template <int D, bool F8 = false>
 struct FwdLayout {
-  static constexpr int kChunks = D / 64;            // 128-byte column chunks per row (>= 1)
-  static constexpr int kChunkBytes = kTile * 128;   // one 128-row chunk
-  static constexpr int kTileBytes = kTile * D * 2;  // one 128 x D 16-bit tile
-  static constexpr bool kWide = D == 256;           // see below
-  static constexpr int kSlots = kWide ? 2 : (D == 128 ? 5 : 10);  // K/V ring slots
+  static constexpr int kElemBytes = F8 ? 1 : 2;
+  static constexpr int kRowBytes = D * kElemBytes;        // one row of Q, K or V
+  static constexpr int kChunks = kRowBytes / 128;         // 128-byte column chunks per row (>= 1)
+  static constexpr int kChunkElems = 128 / kElemBytes;    // elements of one chunk (TMA box width)
+  static constexpr int kChunkBytes = kTile * 128;         // one 128-row chunk
+  static constexpr int kTileBytes = kTile * kRowBytes;    // one 128 x D tile
+  static constexpr int kKeysPerStep = 32 / kElemBytes;    // keys per MMA K step (32 bytes)
+  static constexpr bool kWide = D == 256;                 // see below
+  static constexpr int kSlots = kWide ? 2 : (kTileBytes == 32768 ? 5 : 10);  // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kTileBytes;
   // Exchange between the two softmax warpgroups: row maxima
@@ -80,15 +85,23 @@ struct FwdLayout {
   static constexpr uint32_t kColO = kWide ? 256 : 320;
   static constexpr uint32_t kColL = kColO + D;  // 16 columns: row sums of the 16-bit P (d <= 128)
   static_assert(kWide ? kColO + D <= 512 : kColL + 16 <= 512, "tensor memory budget");
+  static_assert(!F8 || D == 128, "the 8-bit forward is built for d = 128");
 };
 
-template <int D, bool BF16, bool CAUSAL>
+// F8: Q, K, V are E4M3 with per-tensor descale factors.  scale_log2 then
+// carries scale * descale_q * descale_k * log2(e), o_scale = descale_v
+// multiplies O in the epilogue, P is rounded to E4M3 for O += P V (and for
+// its row sums), both products run as kind::f8f6f4, and O is written as bf16
+// (BF16 = true).  The 16-bit kernels ignore o_scale.
+template <int D, bool BF16, bool CAUSAL, bool F8 = false>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o_ptr,
                float* __restrict__ lse_ptr, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H,
-               int Nq, int Nk, int bottom_right, float scale_log2, int problems, int grid_tiles, int group) {
-  using L = FwdLayout<D>;
+               int Nq, int Nk, int bottom_right, float scale_log2, int problems, int grid_tiles, int group,
+               float o_scale) {
+  static_assert(!F8 || BF16, "the 8-bit forward writes bf16");
+  using L = FwdLayout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -189,7 +202,7 @@ __global__ void __launch_bounds__(384, 1)
     tmem_relinquish();
   }
   if (warp == 3) {
-    const uint32_t one2 = BF16 ? 0x3F803F80u : 0x3C003C00u;  // two 16-bit ones
+    const uint32_t one2 = F8 ? 0x38383838u : (BF16 ? 0x3F803F80u : 0x3C003C00u);  // ones (E4M3 or 16-bit)
     uint4* ones = reinterpret_cast<uint4*>(smem + L::kOnesOff);
     for (int i = lane; i < L::kOnesBytes / 16; i += 32) ones[i] = make_uint4(one2, one2, one2, one2);
     fence_proxy_async_smem();
@@ -207,7 +220,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(q_full, L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
-        tma_load_3d(smem + L::kQOff + c * L::kChunkBytes, &tm_q, q_full, c * 64, q0 + qt * kTile, z);
+        tma_load_3d(smem + L::kQOff + c * L::kChunkBytes, &tm_q, q_full, c * L::kChunkElems, q0 + qt * kTile, z);
       // Ring order: K_0, K_1, then V_j, K_{j+2} for j = 0, 1, ...
       int item = 0;
       bool ok = true;
@@ -217,7 +230,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
         uint8_t* dst = smem + L::kRingOff + slot * L::kTileBytes;
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * 64, k0 + tile * kTile, z);
+          tma_load_3d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * L::kChunkElems, k0 + tile * kTile, z);
         ++item;
         return true;
       };
@@ -237,8 +250,9 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs the loop (descriptors stay warp-uniform); one
     // elected lane issues each group of MMAs together with its commits.
-    constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // A = Q (TMEM), B = K K-major
-    constexpr uint32_t kIdPV = idesc_f16(BF16, 128, D, false, true);    // A = P (TMEM), B = V MN-major
+    // A = Q (TMEM), B = K K-major; A = P (TMEM), B = V MN-major.
+    constexpr uint32_t kIdS = F8 ? idesc_e4m3(128, 128, false, false) : idesc_f16(BF16, 128, 128, false, false);
+    constexpr uint32_t kIdPV = F8 ? idesc_e4m3(128, D, false, true) : idesc_f16(BF16, 128, D, false, true);
     const uint32_t ring_base = smem_u32(smem + L::kRingOff);
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
@@ -249,36 +263,50 @@ __global__ void __launch_bounds__(384, 1)
       addr = ring_base + slot * L::kTileBytes;
       return wait_all(&kv_full[slot], (item / L::kSlots) & 1);
     };
-    // S = Q K^T: A = Q in TMEM (8 columns per K step of 16), B = K K-major
-    // (a K step is 32 bytes inside a 128-byte swizzle row).
+    // S = Q K^T: A = Q in TMEM (8 columns per K step of 32 bytes: 16
+    // 16-bit or 32 8-bit values), B = K K-major (a K step is 32 bytes inside
+    // a 128-byte swizzle row).
     const uint64_t qd = sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
     auto issue_s = [&](int b, uint32_t k_addr) {
       const uint64_t kd = sdesc_sw128(k_addr, 16, 1024);
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
+      for (int ks = 0; ks < L::kRowBytes / 32; ++ks) {
         const uint32_t step = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
         if constexpr (L::kWide)  // A = Q in shared memory
           mma_ss(tmem + L::kColS + 128 * b, qd + (step >> 4), kd + (step >> 4), kIdS, ks > 0 ? 1u : 0u);
+        else if constexpr (F8)
+          mma_ts_f8(tmem + L::kColS + 128 * b, tmem + L::kColQ + 8 * ks, kd + (step >> 4), kIdS, ks > 0 ? 1u : 0u);
         else
           mma_ts(tmem + L::kColS + 128 * b, tmem + L::kColQ + 8 * ks, kd + (step >> 4), kIdS, ks > 0 ? 1u : 0u);
       }
     };
-    // O += P V: P in the buffer's TMEM columns (key step ks of 16 keys sits
-    // at 64 (ks / 4) + 8 (ks % 4)), V MN-major (16 rows of 128 bytes); then
-    // L += P 1 against the ones tile (two 256-byte core matrices per step).
-    constexpr uint32_t kIdL = idesc_f16(BF16, 128, 16, false, false);
+    // O += P V: P in the buffer's TMEM columns (a key step of kKeysPerStep
+    // keys takes 8 columns; the keys of warpgroup h start at column 64 h),
+    // V MN-major (kKeysPerStep rows of 128 bytes per step); then L += P 1
+    // against the ones tile (two 256-byte core matrices per step).
+    constexpr uint32_t kIdL = F8 ? idesc_e4m3(128, 16, false, false) : idesc_f16(BF16, 128, 16, false, false);
+    constexpr int kHalfSteps = 64 / L::kKeysPerStep;  // key steps per warpgroup half of a tile
     const uint64_t ones_d = sdesc_noswz(smem_u32(smem + L::kOnesOff), 256, 128);
     auto issue_pv = [&](int b, uint32_t v_addr, bool acc) {
       const uint64_t vd = sdesc_sw128(v_addr, L::kChunkBytes, 1024);
 #pragma unroll
-      for (int ks = 0; ks < kTile / 16; ++ks)
-        mma_ts(tmem + L::kColO, tmem + L::kColS + 128 * b + 64 * (ks >> 2) + 8 * (ks & 3), vd + 128 * ks, kIdPV,
-               (acc || ks > 0) ? 1u : 0u);
+      for (int ks = 0; ks < kTile / L::kKeysPerStep; ++ks) {
+        const uint32_t p_col = tmem + L::kColS + 128 * b + 64 * (ks / kHalfSteps) + 8 * (ks % kHalfSteps);
+        const uint64_t v_step = vd + 8 * L::kKeysPerStep * ks;  // kKeysPerStep rows of 128 bytes, in 16-byte units
+        if constexpr (F8)
+          mma_ts_f8(tmem + L::kColO, p_col, v_step, kIdPV, (acc || ks > 0) ? 1u : 0u);
+        else
+          mma_ts(tmem + L::kColO, p_col, v_step, kIdPV, (acc || ks > 0) ? 1u : 0u);
+      }
       if constexpr (!L::kWide) {
 #pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_ts(tmem + L::kColL, tmem + L::kColS + 128 * b + 64 * (ks >> 2) + 8 * (ks & 3), ones_d + 32 * ks, kIdL,
-                 (acc || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < kTile / L::kKeysPerStep; ++ks) {
+          const uint32_t p_col = tmem + L::kColS + 128 * b + 64 * (ks / kHalfSteps) + 8 * (ks % kHalfSteps);
+          if constexpr (F8)
+            mma_ts_f8(tmem + L::kColL, p_col, ones_d + 32 * ks, kIdL, (acc || ks > 0) ? 1u : 0u);
+          else
+            mma_ts(tmem + L::kColL, p_col, ones_d + 32 * ks, kIdL, (acc || ks > 0) ? 1u : 0u);
+        }
       }
     };
 
@@ -333,20 +361,22 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
 
     // Q -> TMEM: this thread copies its row's half of the head dimension
-    // (16-byte units of the 128-byte swizzled tile) as 16-bit pairs.
+    // (16-byte units of the 128-byte swizzled tile) as 32-bit words of two
+    // 16-bit or four 8-bit values, the lowest K index in the lowest bits.
     bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag));
     if constexpr (!L::kWide) {  // d = 256: Q stays in shared memory
       if (ok) {
-        constexpr int kUnits = D / 16;  // 16-byte units in half a row
-        const uint8_t* qrow = smem + L::kQOff + (D == 128 ? h * L::kChunkBytes : 0) + row * 128;
+        constexpr bool kTwoChunks = L::kRowBytes == 256;  // each warpgroup copies one whole chunk
+        constexpr int kUnits = L::kRowBytes / 32;          // 16-byte units in half a row
+        const uint8_t* qrow = smem + L::kQOff + (kTwoChunks ? h * L::kChunkBytes : 0) + row * 128;
         uint32_t qv[4 * kUnits];
 #pragma unroll
         for (int u = 0; u < kUnits; ++u) {
-          const int unit = (D == 128 ? u : kUnits * h + u) ^ (row & 7);
+          const int unit = (kTwoChunks ? u : kUnits * h + u) ^ (row & 7);
           const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + unit * 16);
           qv[4 * u] = v4.x; qv[4 * u + 1] = v4.y; qv[4 * u + 2] = v4.z; qv[4 * u + 3] = v4.w;
         }
-        if constexpr (D == 128) {
+        if constexpr (kTwoChunks) {
           tmem_st32(t_row + L::kColQ + 32 * h, qv);
         } else {
           tmem_st16(t_row + L::kColQ + 16 * h, qv);
@@ -403,13 +433,28 @@ __global__ void __launch_bounds__(384, 1)
       // the FMA-pipe exponential, since MUFU throughput bounds them otherwise.
       // A row that has seen no key yet (m_run = -inf; causal with off < 0)
       // uses 0: its scores are all -inf, so p = 0 rather than NaN.
-      // (d = 256: the rounded ones are summed here too, in sr.)
+      // (d = 256: the rounded ones are summed here too, in sr.  F8: P is
+      // rounded to E4M3, four keys per 32-bit column, so the 64 keys take
+      // 16 columns; the lazy rescale keeps P <= 2^8, inside E4M3's 448.)
       float2 su[4], sr[4];
 #define ATTN_EXP_STORE()                                                                            \
   {                                                                                                 \
     _Pragma("unroll") for (int i = 0; i < 4; ++i) su[i] = sr[i] = make_float2(0.f, 0.f);            \
     const float m_use = m_run == -INFINITY ? 0.f : m_run;                                           \
     const float2 cx2 = make_float2(cx, cx), negm2 = make_float2(-m_use, -m_use);                    \
+    if constexpr (F8) {                                                                             \
+      uint32_t pk[16];                                                                              \
+      _Pragma("unroll") for (int i = 0; i < 16; ++i) {                                              \
+        const float2 a0 = fma2(make_float2(x[4 * i], x[4 * i + 1]), cx2, negm2);                    \
+        const float2 a1 = fma2(make_float2(x[4 * i + 2], x[4 * i + 3]), cx2, negm2);                \
+        const float2 p0 = make_float2(ex2(a0.x), ex2(a0.y));                                        \
+        const float2 p1 = (i & 1) ? exp2_poly2(a1) : make_float2(ex2(a1.x), ex2(a1.y));             \
+        pk[i] = pack4_e4m3(p0.x, p0.y, p1.x, p1.y);                                                 \
+        su[(2 * i) & 3] = add2(su[(2 * i) & 3], p0);                                                \
+        su[(2 * i + 1) & 3] = add2(su[(2 * i + 1) & 3], p1);                                        \
+      }                                                                                             \
+      tmem_st16(s_col, pk);                                                                         \
+    } else {                                                                                        \
     _Pragma("unroll") for (int c = 0; c < 2; ++c) {                                                 \
       uint32_t pk[16];                                                                              \
       _Pragma("unroll") for (int i = 0; i < 16; ++i) {                                              \
@@ -420,6 +465,7 @@ __global__ void __launch_bounds__(384, 1)
         if constexpr (L::kWide) sr[i & 3] = add2(sr[i & 3], unpack2<BF16>(pk[i]));                  \
       }                                                                                             \
       tmem_st16(s_col + 16 * c, pk);                                                                \
+    }                                                                                               \
     }                                                                                               \
   }
       // Row maximum over both halves of the key tile, exchanged through
@@ -503,7 +549,7 @@ __global__ void __launch_bounds__(384, 1)
         l_tc = lr_run + xsum[(2 + (h ^ 1)) * kTile + row];
       else
         l_tc = __uint_as_float(tmem_ld1(t_row + L::kColL));
-      const float inv = empty ? 0.f : 1.f / l_tc;
+      const float inv = empty ? 0.f : (F8 ? o_scale : 1.f) / l_tc;
       const bool live = qt * kTile + row < nq;  // padding rows of a ragged tile are not stored
       const size_t grow = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile + row;
       uint4* dst = reinterpret_cast<uint4*>(o_ptr + grow * D + (D / 2) * h);

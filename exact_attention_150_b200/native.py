@@ -45,6 +45,8 @@ def load() -> ctypes.CDLL:
     vp, i, f, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int
     lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
     lib.attn_fwd.restype = st
+    lib.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, vp]
+    lib.attn_fwd_fp8.restype = st
     lib.attn_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
@@ -94,6 +96,12 @@ def _check(where: str, status: int) -> None:
 def attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
     """Direct call of attn_fwd with integer device pointers; returns the status."""
     return load().attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, int(causal), dtype, stream)
+
+
+def attn_fwd_fp8(q, k, v, o, lse, B, H, Nq, Nk, d, scale, descale_q, descale_k, descale_v, causal, stream) -> int:
+    """Direct call of attn_fwd_fp8 (E4M3 inputs, bf16 output); returns the status."""
+    return load().attn_fwd_fp8(q, k, v, o, lse, B, H, Nq, Nk, d, scale, descale_q, descale_k, descale_v, int(causal),
+                               stream)
 
 
 def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
@@ -189,6 +197,32 @@ def forward(q, k, v, causal=False, scale: float | None = None, out=None, lse=Non
         stream = torch.cuda.current_stream(q.device).cuda_stream
     _check("attn_fwd", attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                 B, H, Nq, Nk, d, float(scale), causal_code(causal), code, stream))
+    return out, lse
+
+
+def forward_fp8(q, k, v, descale_q: float, descale_k: float, descale_v: float, causal=False,
+                scale: float | None = None, out=None, lse=None, stream=None):
+    """O (bf16), LSE of attention over E4M3 inputs q [B,H,Nq,128], k and v
+    [B,H,Nk,128] (torch.float8_e4m3fn) that stand for descale_x * x."""
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    e4m3 = torch.float8_e4m3fn
+    _check_tensor("q", q, (B, H, Nq, d), e4m3)
+    _check_tensor("k", k, (B, H, Nk, d), e4m3)
+    _check_tensor("v", v, (B, H, Nk, d), e4m3)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check_tensor("out", out, (B, H, Nq, d), torch.bfloat16)
+    _check_tensor("lse", lse, (B, H, Nq), torch.float32)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    _check("attn_fwd_fp8", attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                        B, H, Nq, Nk, d, float(scale), float(descale_q), float(descale_k),
+                                        float(descale_v), causal_code(causal), stream))
     return out, lse
 
 

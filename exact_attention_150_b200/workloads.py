@@ -104,6 +104,34 @@ def draw(B, H, Nq, Nk, d, dtype, seed, input_scale=1.0, with_grad=False, device=
     return tuple(out)
 
 
+# FP8 inputs: the long-context shape (B1 H16 N16384 d128, causal) with Q, K,
+# V as E4M3 codes and one descale factor per tensor, forward only.
+FWD_FP8 = dict(name="fwd_fp8", B=1, H=16, N=16384, d=128, causal=True, seed=1009)
+
+E4M3_MAX = 448.0  # largest finite E4M3 value
+
+
+def draw_fp8(B, H, Nq, Nk, d, seed, device="cpu"):
+    """Seeded E4M3 inputs with per-tensor descale factors.
+
+    Q [B,H,Nq,d], K and V [B,H,Nk,d] are drawn as fp32 i.i.d. N(0, 1) from a
+    CPU generator seeded with ``seed``; each tensor gets descale =
+    max|x| / 448 (1 for an all-zero or empty tensor) and is stored as
+    torch.float8_e4m3fn(x / descale), torch's round-to-nearest-even
+    conversion.  Returns (q8, k8, v8, descale_q, descale_k, descale_v).
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    codes, descales = [], []
+    for n in (Nq, Nk, Nk):
+        t = torch.randn((B, H, n, d), generator=g, dtype=torch.float32)
+        amax = float(t.abs().max()) if t.numel() else 0.0
+        descale = amax / E4M3_MAX if amax > 0 else 1.0
+        codes.append((t / descale).to(torch.float8_e4m3fn).to(device))
+        descales.append(descale)
+    return (*codes, *descales)
+
+
 # Packed variable-length batch: a seeded mix of causal self-attention
 # sequences (lengths uniform in [1024, 16384], the last one cut so that the
 # batch holds 65536 tokens), H = 16, d = 128, bf16, inputs scaled by 0.5.

@@ -107,6 +107,28 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
                      attn_dtype dtype, void* stream);
 
 /*
+ * FP8 forward (page "Flash Attention 是什麼|為何更快又省 VRAM", section
+ * "從 FA-1 到 FA-4": FlashAttention-3 adds an FP8 variant; the page gives no
+ * method, so this is the plain per-tensor-scaled reading).  q, k, v hold
+ * OCP E4M3 bytes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+ * infinities, 0x7F/0xFF NaN, largest finite 448) in the layout of attn_fwd,
+ * and stand for descale_q * q, descale_k * k, descale_v * v.  Writes
+ *   O   = softmax(scale * descale_q * descale_k * q k^T [+ causal mask])
+ *         (descale_v * v), bf16 [B][H][Nq][d];
+ *   LSE = the natural-log row log-sum-exp of those scaled scores, fp32.
+ * Both products run on the 8-bit tensor path: the probabilities are
+ * rounded to E4M3 (round to nearest even, saturating; relative error up
+ * to 2^-4, values below 2^-10 of the running row maximum become 0) before
+ * the product with V, and O is normalised by the sum of the rounded
+ * probabilities.  d must be 128 (ATTN_ERR_UNSUPPORTED otherwise); a
+ * descale factor or scale that is not finite returns ATTN_ERR_INVALID_ARG.
+ * Sizes, masks, empty problems, alignment and errors as for attn_fwd.
+ */
+attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int H, int Nq, int Nk, int d, float scale, float descale_q,
+                         float descale_k, float descale_v, int causal, void* stream);
+
+/*
  * Size in bytes of the device workspace attn_bwd and attn_bwd_deterministic
  * need: an fp32 dQ accumulator [B][H][Nq][d] followed by
  * (128 - Nq % 128) % 128 rows of d floats of padding (a ragged last query

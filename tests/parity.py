@@ -5,6 +5,13 @@ Tolerances (attention parity bar for this library):
   O:   max |O_gpu - O_ref| <= 2e-3 (fp16) or 1e-2 (bf16);
   LSE: max |LSE_gpu - LSE_ref| <= 1e-3;
   dQ, dK, dV: ||G_gpu - G_ref||_F / ||G_ref||_F <= 2e-2.
+FP8 forward (E4M3 inputs, bf16 O), against the oracle's exact attention of
+the descaled inputs: the probabilities are rounded to E4M3 (3 mantissa bits)
+before the product with V, so O is held to ||dO||_F / ||O_ref||_F <= 5e-2
+and max |dO| <= 3e-2 * max |V|, about twice and three times what rounding P
+to E4M3 against the exact row maximum gives on N(0, 1) inputs (2.0-2.5e-2
+and up to 0.9e-2).  LSE is computed from the unrounded probabilities and
+keeps the 1e-3 bar.
 O is stored in 16 bits, and half a unit in the last place of a 16-bit
 number exceeds the O tolerance once |O| >= 4 (bf16) or >= 8 (fp16).  Those
 elements are checked against one unit in the last place of the 16-bit type
@@ -21,6 +28,8 @@ import oracle
 O_TOL = {torch.float16: 2e-3, torch.bfloat16: 1e-2}
 LSE_TOL = 1e-3
 GRAD_TOL = 2e-2
+FP8_O_REL_FRO = 5e-2
+FP8_O_MAX_ABS_OF_VMAX = 3e-2
 _MANT = {torch.float16: 10, torch.bfloat16: 7}
 
 
@@ -97,3 +106,17 @@ def oracle_forward_slices(q, k, v, scale, causal, slices, rows=None):
         outs.append(o)
         lses.append(lse)
     return outs, lses
+
+
+def assert_o_fp8(got, ref, v_max_abs, what=""):
+    """FP8 forward: O within the E4M3 bars above (v_max_abs = max |V| of the
+    descaled values)."""
+    e = rel_fro(got, ref)
+    assert e <= FP8_O_REL_FRO, f"{what}: O relative Frobenius error {e:.3e}"
+    mx = float(np.max(np.abs(got - ref), initial=0.0))
+    assert mx <= FP8_O_MAX_ABS_OF_VMAX * v_max_abs, f"{what}: O max abs err {mx:.3e} (max |V| {v_max_abs:.3e})"
+
+
+def codes(t: torch.Tensor) -> np.ndarray:
+    """The byte codes of a torch.float8_e4m3fn tensor, as a numpy array."""
+    return t.detach().to("cpu").view(torch.uint8).numpy()

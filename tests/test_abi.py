@@ -253,3 +253,30 @@ def test_head_dim_256_is_forward_only(lib):
                 B=1, H=1, Nq=128, Nk=128, d=256, scale=0.1, causal=0, dtype=native.ATTN_BF16, stream=None)
     assert native.attn_bwd_deterministic(**args) == native.ATTN_ERR_UNSUPPORTED
     assert _fwd(d=256, q=None) == native.ATTN_ERR_INVALID_ARG  # validated like any supported d
+
+
+def _fwd_fp8(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, H=1, Nq=128, Nk=128, d=128, scale=0.125,
+                descale_q=1.0, descale_k=1.0, descale_v=1.0, causal=0, stream=None)
+    args.update(kw)
+    return native.attn_fwd_fp8(**args)
+
+
+def test_fp8_forward_validation(lib):
+    for d in (64, 96, 256, 0):
+        assert _fwd_fp8(d=d) == native.ATTN_ERR_UNSUPPORTED
+    for field in ("descale_q", "descale_k", "descale_v", "scale"):
+        assert _fwd_fp8(**{field: float("nan")}) == native.ATTN_ERR_INVALID_ARG
+        assert _fwd_fp8(**{field: float("inf")}) == native.ATTN_ERR_INVALID_ARG
+    for field in ("B", "H", "Nq", "Nk"):
+        assert _fwd_fp8(**{field: -1}) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8(causal=3) == native.ATTN_ERR_INVALID_ARG
+    for name in ("q", "k", "v", "o", "lse"):
+        assert _fwd_fp8(**{name: None}) == native.ATTN_ERR_INVALID_ARG
+        assert _fwd_fp8(**{name: FAKE + 8}) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8(Nk=0) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8(Nq=65535 * 128 + 1) == native.ATTN_ERR_UNSUPPORTED
+    assert _fwd_fp8(B=1 << 16, H=1 << 10, Nq=64 * 128) == native.ATTN_ERR_UNSUPPORTED
+    # Empty problems are valid and touch nothing.
+    assert _fwd_fp8(B=0, q=None, k=None, v=None, o=None, lse=None) == native.ATTN_OK
+    assert _fwd_fp8(Nq=0, q=None, k=None, v=None, o=None, lse=None) == native.ATTN_OK

@@ -44,6 +44,10 @@ int main(void) {
   EXPECT(attn_bwd_varlen(p, p, p, p, (const float*)p, p, p, p, p, p, cu, cu, 2, 1, 300, 300, 200, 200, 256, 0.1f,
                          ATTN_CAUSAL_NONE, ATTN_BF16, 0, NULL) == ATTN_ERR_UNSUPPORTED);
   EXPECT(attn_bwd_varlen_workspace_bytes(2, 1, 300, 200, 64) > 0);
+  EXPECT(attn_fwd_fp8(p, p, p, p, (float*)p, 1, 1, 128, 128, 64, 0.1f, 1.f, 1.f, 1.f, ATTN_CAUSAL_NONE, NULL)
+         == ATTN_ERR_UNSUPPORTED);
+  EXPECT(attn_fwd_fp8(NULL, p, p, p, (float*)p, 1, 1, 128, 128, 128, 0.1f, 1.f, 1.f, 1.f, ATTN_CAUSAL_TOP_LEFT, NULL)
+         == ATTN_ERR_INVALID_ARG);
   EXPECT(attn_bwd_noalloc_max_scratch_bytes() > 0);
   EXPECT(attn_selftest_wait_timeout(0, (int*)p, NULL) == ATTN_ERR_INVALID_ARG);
   printf("ok\n");
