@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload long_ctx] [--seq N] [--no-cpu-baseline] [--e2e-steps E]
-                    [--deterministic] [--varlen]
+                    [--deterministic] [--varlen] [--fp8]
 
 One step is one pass of the whole hot path over one batch of synthetic input:
 the forward kernel, then the three backward kernels (D preprocess, main,
@@ -19,6 +19,10 @@ ranks (an all-reduce of the elapsed time only).
 
 --varlen times a packed variable-length batch instead (attn_fwd_varlen and
 attn_bwd_varlen on a seeded length mix; see workloads.VARLEN_MIX).
+
+--fp8 times the FP8 forward instead (attn_fwd_fp8 on E4M3 Q, K, V with
+per-tensor descales; see workloads.FWD_FP8), against an 8-bit peak of twice
+the measured bf16 peak (the nominal dense ratio).
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on a
 bounded sample of the same workload on the host cores, and prints the same
@@ -63,6 +67,7 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--varlen", action="store_true", help="time a packed variable-length batch")
+    p.add_argument("--fp8", action="store_true", help="time the FP8 (E4M3) forward")
     p.add_argument("--deterministic", action="store_true",
                    help="time the bit-reproducible backward (attn_bwd_deterministic) instead of attn_bwd")
     return p.parse_args(argv)
@@ -508,12 +513,90 @@ def run_varlen(args):
     return 0
 
 
+def run_fp8(args):
+    """The FP8 (E4M3) forward on workloads.FWD_FP8, one forward per step."""
+    import torch
+    rank, world, local_rank = dist_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(device)
+    from exact_attention_150_b200 import native, workloads
+    native.load()
+    w = workloads.FWD_FP8
+    B, H, N, d = w["B"], w["H"], w["N"], w["d"]
+    q8, k8, v8, dq, dk, dv = workloads.draw_fp8(B, H, N, N, d, w["seed"], device=device)
+    scale = 1.0 / math.sqrt(d)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    flops = 4.0 * B * H * N * N * d / (2 if w["causal"] else 1)
+    # Algorithmic bytes: read Q, K, V (1 byte each), write O (bf16) and LSE.
+    nbytes = B * H * N * (3 * d + 2 * d + 4)
+
+    def step():
+        native.forward_fp8(q8, k8, v8, dq, dk, dv, causal=w["causal"], scale=scale, out=o, lse=lse)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize(device)
+    native.device_status()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index) as clocks:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    native.device_status()
+    max_ms = max_over_ranks(start.elapsed_time(end), world, device)
+    peaks, peak_src = load_peaks()
+    # The 8-bit peak: the measured bf16 peak times the nominal 8-bit : 16-bit
+    # ratio of 2 (4.5 / 2.25 PFLOP/s dense).
+    peak8 = 2.0 * float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    fwd_ms = max_ms / args.steps
+    tf = flops / fwd_ms / 1e9
+    line = {
+        "metric": METRIC, "value": aggregate(flops, args.steps, world, max_ms), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": fwd_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic: seeded i.i.d. N(0,1) Q, K, V quantised to E4M3 with per-tensor descales (max|x|/448)",
+        "config": {"workload": f"{w['name']}: fwd causal e4m3 B{B} H{H} N{N} d{d}, bf16 O",
+                   "l2": "no flush: E4M3 Q, K, V of %d MB each" % (B * H * N * d // 2**20),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "fwd_tflops": tf,
+        "kernels": {"fwd_kernel (e4m3)": {"ms": fwd_ms, "tflops": tf, "gbs": nbytes / fwd_ms / 1e6,
+                                          "frac": tf / peak8}},
+        "roofline": {"kernel": "fwd_kernel (e4m3)", "bound": "tensor", "achieved": tf, "peak": peak8,
+                     "unit": "TFLOP/s", "frac": tf / peak8, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained x 2 (nominal e4m3 : bf16 ratio)"},
+        "clocks": clocks.summary(), "e2e": None, "gpu_launches": args.steps,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
     if args.varlen:
         return run_varlen(args)
+    if args.fp8:
+        return run_fp8(args)
     return run_ours(args)
 
 
