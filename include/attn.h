@@ -159,8 +159,8 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      int causal, attn_dtype dtype, void* stream);
 
 /*
- * attn_bwd with a bit-reproducible dQ.  The paper's backward has no such
- * variant; the page "Flash Attention 落地评估" (section 4) raises
+ * attn_bwd with a bit-reproducible dQ.  The backward the pages describe has
+ * no such variant; the page "Flash Attention 落地评估" (section 4) raises
  * reproducibility as a concern, and attn_bwd's dQ depends on the order in
  * which fp32 atomic additions from different key tiles land.  Here the key
  * tiles that reach a query tile add their dQ contributions in ascending
@@ -201,7 +201,7 @@ attn_status attn_bwd_phase(const void* q, const void* k, const void* v, const vo
                            int causal, attn_dtype dtype, int phase, void* stream);
 
 /*
- * attn_bwd without a workspace argument.  The paper has no counterpart: this
+ * attn_bwd without a workspace argument.  The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory when
  * they call -- a plugin running inside another runtime's execution callback,
  * where allocating is not allowed, or a process whose device memory is all
@@ -269,7 +269,7 @@ attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const v
                             int deterministic, void* stream);
 
 /*
- * Self-test of failure detection; the paper has no counterpart.  Launches one
+ * Self-test of failure detection; the pages have no counterpart.  Launches one
  * small kernel on `stream`.  Its first warp waits, through the same bounded
  * mbarrier wait the attention kernels use, on a barrier that nothing ever
  * arrives on, with a limit of `limit_us` microseconds (1 .. 1,000,000).  The
