@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload long_ctx] [--seq N] [--no-cpu-baseline] [--e2e-steps E]
-                    [--deterministic] [--varlen] [--fp8]
+                    [--deterministic] [--varlen] [--fp8] [--e2e-pipelined [--e2e-chunks C]]
 
 One step is one pass of the whole hot path over one batch of synthetic input:
 the forward kernel, then the three backward kernels (D preprocess, main,
@@ -23,6 +23,12 @@ attn_bwd_varlen on a seeded length mix; see workloads.VARLEN_MIX).
 --fp8 times the FP8 forward instead (attn_fwd_fp8 on E4M3 Q, K, V with
 per-tensor descales; see workloads.FWD_FP8), against an 8-bit peak of twice
 the measured bf16 peak (the nominal dense ratio).
+
+The e2e leg copies the step's inputs from pinned host memory, runs it and
+copies every result back, each step.  By default the copies and the calls
+run in order on one stream; --e2e-pipelined runs it through attn_host_step
+instead, which overlaps the copies of one chunk of (batch, head) slices with
+the kernels of another.
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on a
 bounded sample of the same workload on the host cores, and prints the same
@@ -68,6 +74,10 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--varlen", action="store_true", help="time a packed variable-length batch")
     p.add_argument("--fp8", action="store_true", help="time the FP8 (E4M3) forward")
+    p.add_argument("--e2e-pipelined", action="store_true",
+                   help="run the e2e leg through attn_host_step (copies of one chunk of slices overlap the "
+                        "kernels of another); forward+backward workloads only")
+    p.add_argument("--e2e-chunks", type=int, default=4, help="chunks of (batch, head) slices for --e2e-pipelined")
     p.add_argument("--deterministic", action="store_true",
                    help="time the bit-reproducible backward (attn_bwd_deterministic) instead of attn_bwd")
     return p.parse_args(argv)
@@ -374,6 +384,18 @@ def run_ours(args):
             for dst, src in zip(outs_h, (o, lse, dq, dk, dv)):
                 dst.copy_(src, non_blocking=True)
 
+        if args.e2e_pipelined and w.backward:
+            # The same step through attn_host_step: the library copies every
+            # chunk in, runs its kernels and copies its results out, with the
+            # copies of one chunk overlapping the kernels of another.
+            dev_buf = torch.empty(native.attn_host_step_device_bytes(w.B, w.H, w.N, w.N, w.d, args.e2e_chunks),
+                                  dtype=torch.uint8, device=device)
+
+            def e2e_step():  # noqa: F811
+                native.host_step(hq, hk, hv, hdo, causal=w.causal, scale=w.scale, chunks=args.e2e_chunks,
+                                 deterministic=args.deterministic, outs=outs_h, device_buffer=dev_buf,
+                                 device=device, stream=stream.cuda_stream)
+
         e2e_step()
         torch.cuda.synchronize(device)
         if world > 1:
@@ -389,7 +411,9 @@ def run_ours(args):
         native.device_status()
         e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, device)
         e2e = {"value": aggregate(step_flops, args.e2e_steps, world, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "path": (f"attn_host_step, {args.e2e_chunks} chunks" if args.e2e_pipelined and w.backward
+                        else "copies, attn_fwd%s, copies on one stream" % (", attn_bwd" if w.backward else ""))}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -66,6 +66,10 @@ def load() -> ctypes.CDLL:
     lib.attn_bwd_noalloc.restype = st
     lib.attn_bwd_noalloc_max_scratch_bytes.argtypes = []
     lib.attn_bwd_noalloc_max_scratch_bytes.restype = ctypes.c_size_t
+    lib.attn_host_step_device_bytes.argtypes = [i, i, i, i, i, i]
+    lib.attn_host_step_device_bytes.restype = ctypes.c_size_t
+    lib.attn_host_step.argtypes = [vp] * 10 + [ctypes.c_size_t, i, i, i, i, i, f, i, i, i, i, vp]
+    lib.attn_host_step.restype = st
     lib.attn_selftest_wait_timeout.argtypes = [i, vp, vp]
     lib.attn_selftest_wait_timeout.restype = st
     lib.attn_last_device_status.argtypes = [vp]
@@ -134,6 +138,18 @@ def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, Nq, Nk, d, scale, 
 
 def attn_bwd_noalloc_max_scratch_bytes() -> int:
     return int(load().attn_bwd_noalloc_max_scratch_bytes())
+
+
+def attn_host_step_device_bytes(B, H, Nq, Nk, d, chunks) -> int:
+    return int(load().attn_host_step_device_bytes(B, H, Nq, Nk, d, chunks))
+
+
+def attn_host_step(q, k, v, dout, o, lse, dq, dk, dv, device_buffer, device_bytes, B, H, Nq, Nk, d, scale, causal,
+                   dtype, chunks, deterministic, stream) -> int:
+    """Direct call of attn_host_step (host pointers for the tensors, a device
+    pointer for the buffer); returns the status."""
+    return load().attn_host_step(q, k, v, dout, o, lse, dq, dk, dv, device_buffer, device_bytes, B, H, Nq, Nk, d,
+                                 scale, int(causal), dtype, chunks, int(deterministic), stream)
 
 
 def attn_bwd_workspace_bytes(B, H, Nq, Nk, d) -> int:
@@ -352,6 +368,59 @@ def backward_varlen(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seq
                                               int(max_seqlen_k), d, float(scale), causal_code(causal), code,
                                               deterministic, stream))
     return dq, dk, dv
+
+
+def _check_host(name: str, t: torch.Tensor, shape, dtype) -> None:
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def host_step(q, k, v, dout, causal=False, scale: float | None = None, chunks: int = 4,
+              deterministic: bool = False, outs=None, device_buffer=None, device=None, stream=None):
+    """Forward and backward of host-resident q [B,H,Nq,d], k and v
+    [B,H,Nk,d] and dout [B,H,Nq,d] through attn_host_step: the copies of one
+    chunk of slices overlap the kernels of another.  Returns (o, lse, dq, dk,
+    dv) in host memory (page-locked when allocated here).  The call is
+    asynchronous on `stream`: synchronize it before reading the results."""
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    code = _dtype_code(q)
+    for name, t, shp in (("q", q, (B, H, Nq, d)), ("k", k, (B, H, Nk, d)), ("v", v, (B, H, Nk, d)),
+                         ("dout", dout, (B, H, Nq, d))):
+        _check_host(name, t, shp, q.dtype)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if outs is None:
+        outs = (torch.empty((B, H, Nq, d), dtype=q.dtype, pin_memory=True),
+                torch.empty((B, H, Nq), dtype=torch.float32, pin_memory=True),
+                torch.empty((B, H, Nq, d), dtype=q.dtype, pin_memory=True),
+                torch.empty((B, H, Nk, d), dtype=q.dtype, pin_memory=True),
+                torch.empty((B, H, Nk, d), dtype=q.dtype, pin_memory=True))
+    o, lse, dq, dk, dv = outs
+    for name, t, shp, dt in (("o", o, (B, H, Nq, d), q.dtype), ("lse", lse, (B, H, Nq), torch.float32),
+                             ("dq", dq, (B, H, Nq, d), q.dtype), ("dk", dk, (B, H, Nk, d), q.dtype),
+                             ("dv", dv, (B, H, Nk, d), q.dtype)):
+        _check_host(name, t, shp, dt)
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    nbytes = attn_host_step_device_bytes(B, H, Nq, Nk, d, chunks)
+    if device_buffer is None:
+        device_buffer = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+    if not device_buffer.is_cuda or device_buffer.numel() * device_buffer.element_size() < nbytes:
+        raise ValueError(f"device_buffer must be a CUDA buffer of at least {nbytes} bytes")
+    if stream is None:
+        stream = torch.cuda.current_stream(device).cuda_stream
+    _check("attn_host_step", attn_host_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), o.data_ptr(),
+                                            lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                            device_buffer.data_ptr(), device_buffer.numel(), B, H, Nq, Nk, d,
+                                            float(scale), causal_code(causal), code, int(chunks), deterministic,
+                                            stream))
+    return o, lse, dq, dk, dv
 
 
 def selftest_wait_timeout(limit_us: int, result, stream=None) -> int:

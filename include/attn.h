@@ -231,6 +231,40 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
 size_t attn_bwd_noalloc_max_scratch_bytes(void);
 
 /*
+ * Forward and backward of one batch whose tensors live in host memory: the
+ * host-resident form of attn_fwd followed by attn_bwd (or
+ * attn_bwd_deterministic when `deterministic` is non-zero), with the same
+ * shapes, layouts, masks, scale and rounding.
+ *   q_h, k_h, v_h, dout_h  inputs in host memory, [B][H][N][d] 16-bit.
+ *   o_h, dq_h, dk_h, dv_h  outputs in host memory, 16-bit; lse_h [B][H][Nq]
+ *                          float.
+ *   device_buffer          caller-owned device memory of at least
+ *                          attn_host_step_device_bytes(...) bytes, 256-byte
+ *                          aligned: the device copies of every tensor and
+ *                          the backward's workspace.
+ *   chunks                 the B*H slices are processed in this many
+ *                          chunks (>= 1; capped at B*H).
+ * The slices are split into chunks; the host-to-device copies of all chunks
+ * run on an internal stream, each chunk's kernels run on `stream` once its
+ * inputs have landed, and each chunk's results return to the host on a
+ * second internal stream once its kernels are done, so copies of one chunk
+ * overlap the kernels of another.  Everything is asynchronous: `stream`
+ * continues past the call once every result has reached the host, and the
+ * host buffers must stay valid until then.  Host buffers should be
+ * page-locked (cudaHostAlloc / pinned); pageable memory works but its
+ * copies do not overlap.  d must be 64 or 128.  No query rows (B*H*Nq == 0)
+ * writes dK = dV = 0 on the host in stream order; Nq > 0 with Nk = 0
+ * returns ATTN_ERR_INVALID_ARG.  An error return may leave part of the work
+ * enqueued: synchronize the device before reusing the buffers.
+ */
+size_t attn_host_step_device_bytes(int B, int H, int Nq, int Nk, int d, int chunks);
+attn_status attn_host_step(const void* q_h, const void* k_h, const void* v_h, const void* dout_h,
+                           void* o_h, float* lse_h, void* dq_h, void* dk_h, void* dv_h,
+                           void* device_buffer, size_t device_bytes, int B, int H, int Nq, int Nk,
+                           int d, float scale, int causal, attn_dtype dtype, int chunks,
+                           int deterministic, void* stream);
+
+/*
  * Packed variable-length batches.  B sequences of different lengths share
  * one tensor without padding (the pages' "varlen" use: each sequence is an
  * attention problem of its own).  Layout, head-major like the dense calls:

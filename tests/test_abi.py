@@ -280,3 +280,54 @@ def test_fp8_forward_validation(lib):
     # Empty problems are valid and touch nothing.
     assert _fwd_fp8(B=0, q=None, k=None, v=None, o=None, lse=None) == native.ATTN_OK
     assert _fwd_fp8(Nq=0, q=None, k=None, v=None, o=None, lse=None) == native.ATTN_OK
+
+
+def _host_step(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, dout=FAKE, o=FAKE, lse=FAKE, dq=FAKE, dk=FAKE, dv=FAKE,
+                device_buffer=FAKE, device_bytes=1 << 40, B=1, H=4, Nq=300, Nk=300, d=128, scale=0.1, causal=1,
+                dtype=native.ATTN_BF16, chunks=2, deterministic=0, stream=None)
+    args.update(kw)
+    return native.attn_host_step(**args)
+
+
+def _host_step_bytes(B, H, Nq, Nk, d, chunks):
+    # Every region rounded up to 256 bytes: Q, K, V, dO, O, dQ, dK, dV, then
+    # one aligned LSE block per chunk, then one chunk's backward workspace.
+    r = lambda x: (x + 255) // 256 * 256
+    bh = B * H
+    chunks = min(chunks, bh)
+    per = -(-bh // chunks)
+    chunks = -(-bh // per)
+    qb, kb = r(bh * Nq * d * 2), r(bh * Nk * d * 2)
+    return 4 * qb + 4 * kb + r(r(per * Nq * 4) * chunks) + r(native.attn_bwd_workspace_bytes(1, per, Nq, Nk, d))
+
+
+@pytest.mark.parametrize("shape", [(1, 16, 16384, 16384, 128, 4), (2, 3, 300, 129, 64, 4), (1, 5, 7, 9, 128, 3),
+                                   (3, 1, 128, 128, 64, 1), (2, 2, 100, 200, 128, 9)])
+def test_host_step_device_bytes(lib, shape):
+    assert native.attn_host_step_device_bytes(*shape) == _host_step_bytes(*shape)
+
+
+def test_host_step_device_bytes_empty(lib):
+    assert native.attn_host_step_device_bytes(0, 4, 128, 128, 128, 2) == 0
+    assert native.attn_host_step_device_bytes(1, 4, 0, 128, 128, 2) == 0
+    assert native.attn_host_step_device_bytes(1, 4, 128, 128, 128, 0) == 0
+
+
+def test_host_step_validation(lib):
+    assert _host_step(chunks=0) == native.ATTN_ERR_INVALID_ARG
+    for d in (256, 96, 0):
+        assert _host_step(d=d) == native.ATTN_ERR_UNSUPPORTED
+    assert _host_step(dtype=5) == native.ATTN_ERR_UNSUPPORTED
+    assert _host_step(causal=3) == native.ATTN_ERR_INVALID_ARG
+    for field in ("B", "H", "Nq", "Nk"):
+        assert _host_step(**{field: -1}) == native.ATTN_ERR_INVALID_ARG
+    for name in ("q", "k", "v", "dout", "o", "lse", "dq", "dk", "dv", "device_buffer"):
+        assert _host_step(**{name: None}) == native.ATTN_ERR_INVALID_ARG
+    assert _host_step(device_buffer=FAKE + 16) == native.ATTN_ERR_INVALID_ARG  # 256-byte alignment
+    need = native.attn_host_step_device_bytes(1, 4, 300, 300, 128, 2)
+    assert _host_step(device_bytes=need - 1) == native.ATTN_ERR_INVALID_ARG
+    assert _host_step(Nk=0) == native.ATTN_ERR_INVALID_ARG
+    assert _host_step(B=1 << 16, H=1 << 16) == native.ATTN_ERR_UNSUPPORTED
+    assert _host_step(B=0) == native.ATTN_OK  # nothing to do
+    assert _host_step(Nq=0, Nk=0) == native.ATTN_OK
