@@ -413,13 +413,16 @@ def host_step(q, k, v, dout, causal=False, scale: float | None = None, chunks: i
         device_buffer = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
     if not device_buffer.is_cuda or device_buffer.numel() * device_buffer.element_size() < nbytes:
         raise ValueError(f"device_buffer must be a CUDA buffer of at least {nbytes} bytes")
+    if device_buffer.device != device:
+        raise ValueError(f"device_buffer is on {device_buffer.device}, expected {device}")
     if stream is None:
         stream = torch.cuda.current_stream(device).cuda_stream
-    _check("attn_host_step", attn_host_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), o.data_ptr(),
-                                            lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                                            device_buffer.data_ptr(), device_buffer.numel(), B, H, Nq, Nk, d,
-                                            float(scale), causal_code(causal), code, int(chunks), deterministic,
-                                            stream))
+    with torch.cuda.device(device):  # the library's internal copy streams belong to the current device
+        status = attn_host_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), o.data_ptr(),
+                                lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), device_buffer.data_ptr(),
+                                device_buffer.numel(), B, H, Nq, Nk, d, float(scale), causal_code(causal), code,
+                                int(chunks), deterministic, stream)
+    _check("attn_host_step", status)
     return o, lse, dq, dk, dv
 
 

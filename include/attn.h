@@ -255,7 +255,8 @@ size_t attn_bwd_noalloc_max_scratch_bytes(void);
  * copies do not overlap.  d must be 64 or 128.  No query rows (B*H*Nq == 0)
  * writes dK = dV = 0 on the host in stream order; Nq > 0 with Nk = 0
  * returns ATTN_ERR_INVALID_ARG.  An error return may leave part of the work
- * enqueued: synchronize the device before reusing the buffers.
+ * enqueued: synchronize the device before reusing the buffers.  The
+ * current device must own `device_buffer` and `stream`.
  */
 size_t attn_host_step_device_bytes(int B, int H, int Nq, int Nk, int d, int chunks);
 attn_status attn_host_step(const void* q_h, const void* k_h, const void* v_h, const void* dout_h,
