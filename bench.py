@@ -85,6 +85,17 @@ def parse_args(argv=None):
 
 # ---------------------------------------------------------------- helpers
 
+def add_spread(kernels: dict, evs, spans: dict) -> None:
+    """Adds the median and the minimum of each kernel's per-step event times
+    (events a -> b of every step) beside its mean."""
+    for name, (a, b) in spans.items():
+        if name not in kernels or not evs:
+            continue
+        t = [e[a].elapsed_time(e[b]) for e in evs]
+        kernels[name]["ms_median"] = statistics.median(t)
+        kernels[name]["ms_min"] = min(t)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -357,6 +368,9 @@ def run_ours(args):
         dom_name, dom_ms, dom_flops = "bwd_main_kernel", main_ms, w.bwd_flops()
     else:
         dom_name, dom_ms, dom_flops = "fwd_kernel", fwd_ms, w.fwd_flops()
+    spans = {"fwd_kernel": (0, 1), "bwd_deterministic (order counters + 3 kernels)": (1, 2),
+             "bwd_pre_kernel": (1, 2), "bwd_main_kernel": (2, 3), "bwd_post_kernel": (3, 4)}
+    add_spread(kernels, evs, spans)
     for name, kinfo in kernels.items():
         if "tflops" in kinfo:
             kinfo["frac"] = kinfo["tflops"] / peak_sus

@@ -91,3 +91,23 @@ def test_varlen_mix_is_seeded_and_bounded():
     assert q.shape == (2, 8, 8) and cu.tolist() == [0, 3, 8] and cu.dtype == torch.int32
     q2 = workloads.make_varlen_inputs([3, 5], 2, 8, torch.bfloat16, 7)[0]
     assert torch.equal(q, q2)
+
+
+def test_add_spread_median_and_min():
+    import bench
+
+    class Ev:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    # three steps, events at cumulative times; kernel spans (0,1) and (1,2)
+    evs = [[Ev(0.0), Ev(2.0), Ev(7.0)], [Ev(0.0), Ev(1.0), Ev(5.0)], [Ev(0.0), Ev(4.0), Ev(6.0)]]
+    kernels = {"a": {"ms": 0.0}, "b": {"ms": 0.0}}
+    bench.add_spread(kernels, evs, {"a": (0, 1), "b": (1, 2), "missing": (0, 2)})
+    assert kernels["a"]["ms_median"] == 2.0 and kernels["a"]["ms_min"] == 1.0
+    assert kernels["b"]["ms_median"] == 4.0 and kernels["b"]["ms_min"] == 2.0
+    assert "missing" not in kernels
+    bench.add_spread(kernels, [], {"a": (0, 1)})  # no steps: nothing added, no error
