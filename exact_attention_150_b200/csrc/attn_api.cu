@@ -13,6 +13,7 @@
 #include "attn.h"
 #include "bwd_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "trace.h"
 
 namespace {
 
@@ -400,6 +401,7 @@ extern "C" {
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
                      int d, float scale, int causal, attn_dtype dtype, void* stream) {
+  attn::TraceRange trace("attn_fwd");
   const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
   if (B == 0 || H == 0 || Nq == 0) return ATTN_OK;  // no query rows: nothing to write
@@ -413,6 +415,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
 attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
                          int Nk, int d, float scale, float descale_q, float descale_k, float descale_v, int causal,
                          void* stream) {
+  attn::TraceRange trace("attn_fwd_fp8");
   const attn_status cs = check_common(B, H, Nq, Nk, d, causal, ATTN_BF16);
   if (cs != ATTN_OK) return cs;
   if (d != 128) return ATTN_ERR_UNSUPPORTED;
@@ -438,6 +441,7 @@ attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, f
 attn_status attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
                             const int* cu_seqlens_k, int B, int H, int total_q, int total_k, int max_seqlen_q,
                             int max_seqlen_k, int d, float scale, int causal, attn_dtype dtype, void* stream) {
+  attn::TraceRange trace("attn_fwd_varlen");
   const attn_status cs = check_varlen(B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
   if (B == 0 || H == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;  // no query rows
@@ -476,6 +480,7 @@ attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const v
                             const int* cu_seqlens_k, int B, int H, int total_q, int total_k, int max_seqlen_q,
                             int max_seqlen_k, int d, float scale, int causal, attn_dtype dtype, int deterministic,
                             void* stream) {
+  attn::TraceRange trace("attn_bwd_varlen");
   const attn_status cs = check_varlen(B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
   if (d == 256) return ATTN_ERR_UNSUPPORTED;  // forward only
@@ -535,6 +540,7 @@ namespace {
 attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                      void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk, int d, float scale,
                      int causal, attn_dtype dtype, int phase, bool det, void* stream) {
+  attn::TraceRange trace(det ? "attn_bwd_deterministic" : "attn_bwd");
   if (phase < ATTN_BWD_ALL || phase > ATTN_BWD_CONVERT) return ATTN_ERR_INVALID_ARG;
   const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
@@ -585,6 +591,7 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
 size_t attn_bwd_noalloc_max_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 attn_status attn_selftest_wait_timeout(int limit_us, int* result, void* stream) {
+  attn::TraceRange trace("attn_selftest_wait_timeout");
   if (limit_us < 1 || limit_us > 1000000 || !result) return ATTN_ERR_INVALID_ARG;
   attn::selftest_wait_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<unsigned long long>(limit_us) * 1000ull, result);

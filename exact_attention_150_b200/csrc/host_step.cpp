@@ -16,6 +16,7 @@
 #include <vector>
 
 #include "attn.h"
+#include "trace.h"
 
 namespace {
 
@@ -133,6 +134,7 @@ attn_status attn_host_step(const void* q_h, const void* k_h, const void* v_h, co
                            float* lse_h, void* dq_h, void* dk_h, void* dv_h, void* device_buffer,
                            size_t device_bytes, int B, int H, int Nq, int Nk, int d, float scale, int causal,
                            attn_dtype dtype, int chunks, int deterministic, void* stream) {
+  attn::TraceRange trace("attn_host_step");
   if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d < 0 || chunks < 1) return ATTN_ERR_INVALID_ARG;
   if (causal != ATTN_CAUSAL_NONE && causal != ATTN_CAUSAL_TOP_LEFT && causal != ATTN_CAUSAL_BOTTOM_RIGHT)
     return ATTN_ERR_INVALID_ARG;
