@@ -199,7 +199,9 @@ class ClockSampler:
 
 def oracle_sample_run(w, q, k, v, do, rows_count: int):
     """One fp64 oracle forward + backward on the last `rows_count` query rows
-    of head (0, 0) against all keys.  Returns (seconds, flops, description)."""
+    of head (0, 0) against all keys.  Returns (seconds, flops, description,
+    (r0, O, LSE, dQ)): the oracle's outputs for those rows, which depend on
+    no other query row."""
     import oracle
     import torch
     f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
@@ -208,12 +210,44 @@ def oracle_sample_run(w, q, k, v, do, rows_count: int):
     qs, dos = f64(q[0, 0, r0:]), f64(do[0, 0, r0:])
     ks, vs = f64(k[0, 0]), f64(v[0, 0])
     t0 = time.perf_counter()
-    oracle.forward(qs, ks, vs, w.scale, w.causal, q_offset=r0)
-    oracle.backward(qs, ks, vs, dos, w.scale, w.causal, q_offset=r0)
+    o, lse, _ = oracle.forward(qs, ks, vs, w.scale, w.causal, q_offset=r0)
+    dq, _, _ = oracle.backward(qs, ks, vs, dos, w.scale, w.causal, q_offset=r0)
     dt = time.perf_counter() - t0
     desc = (f"fp64 oracle forward+backward of query rows [{r0},{n}) of head (0,0) against all {n} keys "
             f"({rows_count} of {w.B * w.H * n} rows of the workload)")
-    return dt, sample_flops(w, range(r0, n)), desc
+    return dt, sample_flops(w, range(r0, n)), desc, (r0, o, lse, dq)
+
+
+# Parity bars: max-abs O (by dtype), max-abs LSE, relative Frobenius dQ.
+PARITY_TOL = {"o": {"bf16": 1e-2, "fp16": 2e-3}, "lse": 1e-3, "dq": 2e-2}
+
+
+def sample_parity(w, ref, o, lse, dq):
+    """Errors of the timed run's outputs (device tensors [B,H,N,...]) against
+    the oracle's outputs `ref` from oracle_sample_run; dq None when the
+    workload has no backward."""
+    import numpy as np
+    import torch
+    r0, o_ref, lse_ref, dq_ref = ref
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    got_o, got_l = f64(o[0, 0, r0:]), f64(lse[0, 0, r0:])
+    fin = np.isfinite(lse_ref)
+    out = {"rows": f"query rows [{r0},{r0 + len(lse_ref)}) of head (0,0)",
+           "o_max_abs_err": float(np.max(np.abs(got_o - o_ref), initial=0.0)),
+           "lse_max_abs_err": float(np.max(np.abs(got_l[fin] - lse_ref[fin]), initial=0.0)),
+           "tol": {"o": PARITY_TOL["o"][w.dtype], "lse": PARITY_TOL["lse"]}}
+    ok = out["o_max_abs_err"] <= out["tol"]["o"] and out["lse_max_abs_err"] <= out["tol"]["lse"]
+    if dq is not None:
+        den = float(np.linalg.norm(dq_ref))
+        out["dq_rel_fro_err"] = float(np.linalg.norm(f64(dq[0, 0, r0:]) - dq_ref)) / (den if den > 0 else 1.0)
+        out["tol"]["dq"] = PARITY_TOL["dq"]
+        ok = ok and out["dq_rel_fro_err"] <= PARITY_TOL["dq"]
+    out["within_tol"] = bool(ok)
+    for key in ("o_max_abs_err", "lse_max_abs_err", "dq_rel_fro_err"):  # keep the line strict JSON
+        if key in out and not math.isfinite(out[key]):
+            out[key] = "non-finite"
+            out["within_tol"] = False
+    return out
 
 
 def blas_threads() -> int:
@@ -248,7 +282,7 @@ def run_reference(args):
     times, flops = [], 0.0
     desc = ""
     for i in range(args.warmup + args.steps):
-        dt, fl, desc = oracle_sample_run(w, q, k, v, do, rows)
+        dt, fl, desc, _ = oracle_sample_run(w, q, k, v, do, rows)
         if i >= args.warmup:
             times.append(dt)
             flops = fl
@@ -430,9 +464,12 @@ def run_ours(args):
                         else "copies, attn_fwd%s, copies on one stream" % (", attn_bwd" if w.backward else ""))}
 
     cpu = None
+    parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, fl, desc = oracle_sample_run(w, q_h, k_h, v_h, do_h, min(4096, w.N))
+        dt, fl, desc, ref = oracle_sample_run(w, q_h, k_h, v_h, do_h, min(4096, w.N))
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": desc}
+        # The same oracle rows against this run's outputs.
+        parity = sample_parity(w, ref, o, lse, dq if w.backward else None)
 
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -454,6 +491,7 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "cpu_baseline": cpu,
+        "parity": parity,
     }
     print(json.dumps(line), flush=True)
     return 0

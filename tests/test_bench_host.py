@@ -111,3 +111,46 @@ def test_add_spread_median_and_min():
     assert kernels["b"]["ms_median"] == 4.0 and kernels["b"]["ms_min"] == 2.0
     assert "missing" not in kernels
     bench.add_spread(kernels, [], {"a": (0, 1)})  # no steps: nothing added, no error
+
+
+def test_sample_parity_against_the_oracle_rows():
+    # The oracle's sampled rows checked against outputs made by the oracle on
+    # the whole problem: zero error; a perturbed O or dQ is reported.
+    import numpy as np
+    import torch
+
+    import bench
+    import oracle
+    from exact_attention_150_b200 import workloads
+    w = workloads.Workload("t", 1, 2, 300, 64, "bf16", True, True, 77)
+    q, k, v, do = workloads.make_inputs(w, with_grad=True)
+    dt, fl, desc, ref = bench.oracle_sample_run(w, q, k, v, do, 100)
+    f64 = lambda t: t.to(torch.float64).numpy()
+    o, lse, _ = oracle.forward(f64(q), f64(k), f64(v), w.scale, True)
+    dq, _, _ = oracle.backward(f64(q), f64(k), f64(v), f64(do), w.scale, True)
+    o_t, lse_t, dq_t = (torch.from_numpy(np.ascontiguousarray(x)) for x in (o, lse, dq))
+    good = bench.sample_parity(w, ref, o_t, lse_t, dq_t)
+    assert good["within_tol"] and good["o_max_abs_err"] < 1e-9 and good["dq_rel_fro_err"] < 1e-9
+    assert good["rows"] == "query rows [200,300) of head (0,0)"
+    o_t[0, 0, 250, 3] += 0.5
+    bad = bench.sample_parity(w, ref, o_t, lse_t, None)
+    assert not bad["within_tol"] and abs(bad["o_max_abs_err"] - 0.5) < 1e-9 and "dq_rel_fro_err" not in bad
+    import json
+    json.dumps(bad, allow_nan=False)
+
+
+def test_sample_parity_non_finite_output_stays_strict_json():
+    import json
+
+    import torch
+
+    import bench
+    from exact_attention_150_b200 import workloads
+    w = workloads.Workload("t", 1, 1, 130, 64, "fp16", False, False, 78)
+    q, k, v, do = workloads.make_inputs(w, with_grad=True)
+    _, _, _, ref = bench.oracle_sample_run(w, q, k, v, do, 10)
+    o = torch.full((1, 1, 130, 64), float("nan"))
+    lse = torch.zeros(1, 1, 130)
+    out = bench.sample_parity(w, ref, o, lse, None)
+    assert out["o_max_abs_err"] == "non-finite" and out["within_tol"] is False
+    json.dumps(out, allow_nan=False)
