@@ -291,6 +291,21 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
               : dispatch_fwd_causal<128, false>(causal, mq, mk, mv, o, lse, pb, sl2, st);
 }
 
+// The FP8 forward launch shared by attn_fwd_fp8 and attn_fwd_fp8_varlen (d = 128).
+attn_status fwd_fp8_impl(const void* q, const void* k, const void* v, void* o, float* lse, const Problem& pb,
+                         float scale, float descale_q, float descale_k, float descale_v, int causal, void* stream) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, pb.slabs, pb.rows_q, 128, true, true) ||
+      !make_map(&mk, k, pb.slabs, pb.rows_k, 128, true, true) ||
+      !make_map(&mv, v, pb.slabs, pb.rows_k, 128, true, true))
+    return ATTN_ERR_CUDA;
+  // The scores are scale * (descale_q q) . (descale_k k): one factor, in log2 units.
+  const float sl2 = scale * descale_q * descale_k * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return causal ? launch_fwd<128, true, true, true>(mq, mk, mv, o, lse, pb, sl2, st, descale_v)
+                : launch_fwd<128, true, false, true>(mq, mk, mv, o, lse, pb, sl2, st, descale_v);
+}
+
 template <int D, bool BF16>
 attn_status dispatch_bwd_causal(int causal, bool det, const CUtensorMap& mq, const CUtensorMap& mk,
                                 const CUtensorMap& mv, const CUtensorMap& mdo, const void* o, const void* dout,
@@ -426,16 +441,33 @@ attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, f
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return ATTN_ERR_INVALID_ARG;
-  const Problem pb = dense_problem(B, H, Nq, Nk, causal);
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, pb.slabs, pb.rows_q, d, true, true) || !make_map(&mk, k, pb.slabs, pb.rows_k, d, true, true) ||
-      !make_map(&mv, v, pb.slabs, pb.rows_k, d, true, true))
-    return ATTN_ERR_CUDA;
-  // The scores are scale * (descale_q q) . (descale_k k): one factor, in log2 units.
-  const float sl2 = scale * descale_q * descale_k * 1.4426950408889634f;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return causal ? launch_fwd<128, true, true, true>(mq, mk, mv, o, lse, pb, sl2, st, descale_v)
-                : launch_fwd<128, true, false, true>(mq, mk, mv, o, lse, pb, sl2, st, descale_v);
+  return fwd_fp8_impl(q, k, v, o, lse, dense_problem(B, H, Nq, Nk, causal), scale, descale_q, descale_k, descale_v,
+                      causal, stream);
+}
+
+attn_status attn_fwd_fp8_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                                const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int total_q,
+                                int total_k, int max_seqlen_q, int max_seqlen_k, int d, float scale, float descale_q,
+                                float descale_k, float descale_v, int causal, void* stream) {
+  attn::TraceRange trace("attn_fwd_fp8_varlen");
+  const attn_status cs = check_varlen(B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, d, causal, ATTN_BF16);
+  if (cs != ATTN_OK) return cs;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!std::isfinite(descale_q) || !std::isfinite(descale_k) || !std::isfinite(descale_v) || !std::isfinite(scale))
+    return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;  // no query rows
+  if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (total_k == 0)  // no sequence has keys: O = 0, LSE = -inf (the query tensor stands in for K and V)
+    return fwd_fp8_impl(q, q, q, o, lse,
+                        varlen_problem(B, H, total_q, 1, max_seqlen_q, 1, cu_seqlens_q, cu_seqlens_k, causal), scale,
+                        descale_q, descale_k, descale_v, causal, stream);
+  return fwd_fp8_impl(q, k, v, o, lse,
+                      varlen_problem(B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, cu_seqlens_q, cu_seqlens_k,
+                                     causal),
+                      scale, descale_q, descale_k, descale_v, causal, stream);
 }
 
 attn_status attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,

@@ -47,6 +47,8 @@ def load() -> ctypes.CDLL:
     lib.attn_fwd.restype = st
     lib.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, vp]
     lib.attn_fwd_fp8.restype = st
+    lib.attn_fwd_fp8_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, f, f, f, i, vp]
+    lib.attn_fwd_fp8_varlen.restype = st
     lib.attn_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
@@ -106,6 +108,13 @@ def attn_fwd_fp8(q, k, v, o, lse, B, H, Nq, Nk, d, scale, descale_q, descale_k, 
     """Direct call of attn_fwd_fp8 (E4M3 inputs, bf16 output); returns the status."""
     return load().attn_fwd_fp8(q, k, v, o, lse, B, H, Nq, Nk, d, scale, descale_q, descale_k, descale_v, int(causal),
                                stream)
+
+
+def attn_fwd_fp8_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, total_q, total_k, max_q, max_k, d, scale, descale_q,
+                        descale_k, descale_v, causal, stream) -> int:
+    """Direct call of attn_fwd_fp8_varlen; returns the status."""
+    return load().attn_fwd_fp8_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, total_q, total_k, max_q, max_k, d, scale,
+                                      descale_q, descale_k, descale_v, int(causal), stream)
 
 
 def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
@@ -332,6 +341,38 @@ def forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_s
                                               cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, H, total_q,
                                               total_k, int(max_seqlen_q), int(max_seqlen_k), d, float(scale),
                                               causal_code(causal), code, stream))
+    return out, lse
+
+
+def forward_fp8_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                       descale_q: float, descale_k: float, descale_v: float, causal=False,
+                       scale: float | None = None, out=None, lse=None, stream=None):
+    """O (bf16), LSE of a packed variable-length batch of E4M3 inputs: q
+    [H, total_q, 128], k and v [H, total_k, 128] (torch.float8_e4m3fn)."""
+    H, total_q, d = q.shape
+    total_k = k.shape[1]
+    B = cu_seqlens_q.shape[0] - 1
+    e4m3 = torch.float8_e4m3fn
+    _check_tensor("q", q, (H, total_q, d), e4m3)
+    _check_tensor("k", k, (H, total_k, d), e4m3)
+    _check_tensor("v", v, (H, total_k, d), e4m3)
+    _check_cu("cu_seqlens_q", cu_seqlens_q, B)
+    _check_cu("cu_seqlens_k", cu_seqlens_k, B)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((H, total_q, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    _check_tensor("out", out, (H, total_q, d), torch.bfloat16)
+    _check_tensor("lse", lse, (H, total_q), torch.float32)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    _check("attn_fwd_fp8_varlen",
+           attn_fwd_fp8_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                               cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, H, total_q, total_k,
+                               int(max_seqlen_q), int(max_seqlen_k), d, float(scale), float(descale_q),
+                               float(descale_k), float(descale_v), causal_code(causal), stream))
     return out, lse
 
 

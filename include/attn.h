@@ -129,6 +129,17 @@ attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, f
                          float descale_k, float descale_v, int causal, void* stream);
 
 /*
+ * FP8 forward of a packed variable-length batch: attn_fwd_varlen's layout,
+ * offsets, masks and empty-sequence rules with attn_fwd_fp8's E4M3 inputs,
+ * per-tensor descale factors, bf16 O and rounding.  d must be 128.
+ */
+attn_status attn_fwd_fp8_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                                const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H,
+                                int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                                float scale, float descale_q, float descale_k, float descale_v,
+                                int causal, void* stream);
+
+/*
  * Size in bytes of the device workspace attn_bwd and attn_bwd_deterministic
  * need: an fp32 dQ accumulator [B][H][Nq][d] followed by
  * (128 - Nq % 128) % 128 rows of d floats of padding (a ragged last query

@@ -52,3 +52,40 @@ def test_fp8_forward_empty_and_invalid():
     with pytest.raises(native.AttnError):
         native.forward_fp8(k[..., :64].contiguous(), k[..., :64].contiguous(), k[..., :64].contiguous(), 1.0, 1.0,
                            1.0)
+
+
+@pytest.mark.parametrize("causal", [False, True, "bottom_right"])
+def test_fp8_forward_varlen(causal):
+    # Packed [H, total, 128] E4M3 batch; each sequence against the oracle on
+    # its own rows (empty and one-token sequences included).
+    import oracle
+    from tests import parity
+    lens_q, lens_k = [300, 1, 0, 129, 257], [200, 5, 40, 0, 257]
+    H = 2
+    tq, tk = sum(lens_q), sum(lens_k)
+    q8, k8, v8, dq, dk, dv = workloads.draw_fp8(1, H, tq, tk, 128, 3300)
+    q8, k8, v8 = (t[0].to(DEV) for t in (q8, k8, v8))
+    cu = lambda lens: torch.tensor([0] + torch.tensor(lens).cumsum(0).tolist(), dtype=torch.int32, device=DEV)
+    scale = 1 / math.sqrt(128)
+    o, lse = native.forward_fp8_varlen(q8, k8, v8, cu(lens_q), cu(lens_k), max(lens_q), max(lens_k), dq, dk, dv,
+                                       causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    native.device_status()
+    o, lse = o.cpu(), lse.cpu()
+    qc, kc, vc = (parity.codes(t) for t in (q8, k8, v8))
+    a = b = 0
+    for nq, nk in zip(lens_q, lens_k):
+        oc, off = parity.oracle_mask(causal, nq, nk)
+        for h in range(H):
+            if nq == 0:
+                continue
+            if nk == 0:
+                assert torch.all(o[h, a:a + nq].float() == 0) and torch.all(torch.isinf(lse[h, a:a + nq]))
+                continue
+            ref, lref = oracle.forward_fp8(qc[h, a:a + nq], kc[h, b:b + nk], vc[h, b:b + nk], dq, dk, dv, scale, oc,
+                                           q_offset=off)
+            vmax = float(np.abs(dv * oracle.e4m3_decode(vc[h, b:b + nk])).max())
+            parity.assert_o_fp8(parity.f64(o[h, a:a + nq]), ref, vmax, f"seq {nq}x{nk} head {h}")
+            parity.assert_lse(parity.f64(lse[h, a:a + nq]), lref, f"seq {nq}x{nk} head {h}")
+        a += nq
+        b += nk

@@ -331,3 +331,28 @@ def test_host_step_validation(lib):
     assert _host_step(B=1 << 16, H=1 << 16) == native.ATTN_ERR_UNSUPPORTED
     assert _host_step(B=0) == native.ATTN_OK  # nothing to do
     assert _host_step(Nq=0, Nk=0) == native.ATTN_OK
+
+
+def _fwd_fp8_varlen(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, cu_q=FAKE, cu_k=FAKE, B=2, H=3, total_q=300, total_k=400,
+                max_q=200, max_k=300, d=128, scale=0.125, descale_q=1.0, descale_k=1.0, descale_v=1.0, causal=0,
+                stream=None)
+    args.update(kw)
+    return native.attn_fwd_fp8_varlen(**args)
+
+
+def test_fp8_varlen_validation(lib):
+    for field in ("B", "H", "total_q", "total_k", "max_q", "max_k"):
+        assert _fwd_fp8_varlen(**{field: -1}) == native.ATTN_ERR_INVALID_ARG
+    for d in (64, 256, 96):
+        assert _fwd_fp8_varlen(d=d) == native.ATTN_ERR_UNSUPPORTED
+    for field in ("descale_q", "descale_k", "descale_v", "scale"):
+        assert _fwd_fp8_varlen(**{field: float("nan")}) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8_varlen(causal=3) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8_varlen(max_q=65535 * 128 + 1) == native.ATTN_ERR_UNSUPPORTED
+    for name in ("q", "k", "v", "o", "lse", "cu_q", "cu_k"):
+        assert _fwd_fp8_varlen(**{name: None}) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8_varlen(cu_k=FAKE + 2) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8_varlen(q=FAKE + 8) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd_fp8_varlen(B=0) == native.ATTN_OK
+    assert _fwd_fp8_varlen(total_q=0) == native.ATTN_OK
