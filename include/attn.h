@@ -18,10 +18,13 @@
  * ---------------------------------------
  * Layout.  Q, O, dO, dQ are contiguous [B][H][Nq][d]; K, V, dK, dV are
  *   contiguous [B][H][Nk][d]; LSE is contiguous [B][H][Nq] float.  Element
- *   type is fp16 or bf16 (attn_dtype) for every 16-bit tensor of one call.
+ *   type is fp16 or bf16 (attn_dtype) for every 16-bit tensor of one call;
+ *   the FP8 calls take E4M3 Q, K, V and write bf16 O.
  * Memory.  Every pointer is a DEVICE pointer on the current CUDA device,
- *   16-byte aligned, allocated and owned by the caller.  The library keeps no
- *   allocation of its own between calls.
+ *   16-byte aligned, allocated and owned by the caller, except the tensors
+ *   of attn_host_step, which live in host memory.  The library keeps no
+ *   allocation of its own between calls, except attn_bwd_noalloc's fixed
+ *   scratch array and attn_host_step's two copy streams per device.
  * Stream.  `stream` is a cudaStream_t (NULL = legacy default stream).  Every
  *   call only enqueues work on it and returns without synchronising.
  * Mask.  `causal` is an attn_causal value; anything else returns
