@@ -63,6 +63,8 @@ struct Plan {
 bool make_plan(int B, int H, int Nq, int Nk, int d, int chunks, Plan* p) {
   p->bh = static_cast<long long>(B) * H;
   if (p->bh <= 0 || p->bh > 0x7fffffffLL || Nq <= 0 || Nk <= 0 || d <= 0 || chunks <= 0) return false;
+  // The row bounds of the attention calls; they also keep the sizes below far from size_t overflow.
+  if (p->bh * Nq > (1LL << 40) || p->bh * Nk > (1LL << 40)) return false;
   p->chunks = static_cast<int>(p->bh < chunks ? p->bh : chunks);
   p->per_chunk = (p->bh + p->chunks - 1) / p->chunks;
   p->chunks = static_cast<int>((p->bh + p->per_chunk - 1) / p->per_chunk);  // no empty chunk

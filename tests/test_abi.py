@@ -312,6 +312,8 @@ def test_host_step_device_bytes_empty(lib):
     assert native.attn_host_step_device_bytes(0, 4, 128, 128, 128, 2) == 0
     assert native.attn_host_step_device_bytes(1, 4, 0, 128, 128, 2) == 0
     assert native.attn_host_step_device_bytes(1, 4, 128, 128, 128, 0) == 0
+    # Past the attention calls' row bounds (B*H*N <= 2^40): no size, rather than a wrapped one.
+    assert native.attn_host_step_device_bytes(1 << 16, 1 << 14, 1, (1 << 23) - 1, 128, 4) == 0
 
 
 def test_host_step_validation(lib):
