@@ -36,15 +36,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3D view [slabs][N][d] of a contiguous 16-bit tensor (a slab is one
-// (batch, head) slice of a dense batch, or one head of a packed
-// variable-length batch), read in boxes of 64 columns (128 bytes) x 128 rows
-// of one slab with the 128-byte swizzle the MMA descriptors expect.  Rows
-// past N read as zeros, so a ragged last tile never touches the next slab.
+// 3D view [slabs][N][d] of a contiguous 16-bit (or, with e4m3, 8-bit)
+// tensor (a slab is one (batch, head) slice of a dense batch, or one head of
+// a packed variable-length batch), read in boxes 128 bytes wide (64 16-bit
+// or 128 8-bit columns) x 128 rows of one slab, with the 128-byte swizzle
+// the MMA descriptors expect.  Rows past N read as zeros, so a ragged last
+// tile never touches the next slab.
 bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16, bool e4m3 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  // Boxes are 128 bytes wide (64 16-bit or 128 8-bit elements) by 128 rows.
   const cuuint64_t eb = e4m3 ? 1 : 2;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * eb, static_cast<cuuint64_t>(N) * d * eb};
