@@ -604,6 +604,7 @@ extern "C" {
 attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                              const void* dout, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d,
                              float scale, int causal, attn_dtype dtype, void* stream) {
+  attn::TraceRange trace("attn_bwd_noalloc");
   const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
   if (attn_bwd_workspace_bytes(B, H, Nq, Nk, d) > kNoAllocScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
@@ -650,6 +651,7 @@ const char* attn_status_string(attn_status s) {
     case ATTN_ERR_TIMEOUT: return "device wait timed out";
     case ATTN_ERR_SMEM: return "kernel found less shared memory than its tiles need";
     case ATTN_ERR_SCRATCH_LIMIT: return "problem needs more scratch than attn_bwd_noalloc's fixed 72 MiB array";
+    case ATTN_ERR_RANGE: return "fp16 backward: a per-query term |LSE/scale| or |D| reached 2^31";
   }
   return "unknown status";
 }

@@ -45,9 +45,10 @@
 // tile's P pass while dK and dQ run on the tensor core.
 // The per-query terms -LSE_i / scale and -D_i enter through one extra K step
 // of 16 in the S^T and dP^T products: the A operand is a constant tile that
-// selects them ([1,1,0,...] or [0,0,1,1,0,...] in every key row) and the B
-// operand holds, per query row, each term as a 16-bit high part plus a
-// 16-bit remainder.  The softmax warps thus need no per-query data at all.
+// selects them ([w0,w1,w2,w3,0,...] or [0,0,0,0,w0,w1,w2,w3,0,...] in every
+// key row) and the B operand holds, per query row, each term as four 16-bit
+// pieces whose weighted sum is the term (see ext_pieces).  The softmax warps
+// thus need no per-query data at all.
 // Warp 3 writes that B block for the next query tile while the current one
 // is in use (single buffer, released by the dP^T product).
 #pragma once
@@ -71,7 +72,7 @@ struct BwdLayout {
   static constexpr int kDSBytes = kBwdTile * kBwdTile * 2;
   // Extra K step: A_ext = two unswizzled 8x16-byte core matrices per term
   // (selector row, zeros), read with a zero row-group stride; B_ext = 128
-  // query rows x 16 bytes [s_hi, s_lo, d_hi, d_lo, 0, 0, 0, 0].
+  // query rows x 16 bytes [s0, s1, s2, s3, d0, d1, d2, d3].
   static constexpr int kAExtOff = kDSOff + kDSBytes;
   static constexpr int kAExtBytes = 4 * 128;
   static constexpr int kBExtOff = kAExtOff + kAExtBytes;
@@ -125,6 +126,57 @@ __global__ void __launch_bounds__(256)
     // stand-in keeps the extra MMA K step free of inf - inf.
     nlse2[row] = lse[row] == -INFINITY ? 0.f : -lse[row] * 1.4426950408889634074f;
   }
+}
+
+// Weight of piece i of a per-query term in the extra K step.  bf16 has
+// fp32's exponent range: three pieces of weight 1 (v = b0 + b1 + b2, the
+// remainder of each rounding carried by the next, 24 bits in all).  fp16 tops
+// out at 65504, so its four pieces sit on a ladder of powers of two 11 bits
+// apart, each holding what the one above left:
+//   v = 2^15 b0 + 2^5 b1 + 2^-6 b2 + 2^-14 b3,
+// exact to about 2^-28 and valid for |v| < 2^31 (b0 <= 65504).  Every weight
+// is a 16-bit normal number, and every product with it is exact in fp32.
+template <bool BF16>
+__device__ __forceinline__ float ext_weight(int i) {
+  if constexpr (BF16) return i < 3 ? 1.f : 0.f;
+  return i == 0 ? 32768.f : (i == 1 ? 32.f : (i == 2 ? 0.015625f : 6.103515625e-05f));
+}
+// 1 / ext_weight(i), exact (powers of two).
+template <bool BF16>
+__device__ __forceinline__ float ext_inv_weight(int i) {
+  if constexpr (BF16) return 1.f;
+  return i == 0 ? 3.0517578125e-05f : (i == 1 ? 0.03125f : (i == 2 ? 64.f : 16384.f));
+}
+// Largest |v| the pieces represent: 2^31 for fp16; bf16 covers every finite
+// fp32 value.
+template <bool BF16>
+__device__ __forceinline__ bool ext_in_range(float v) {
+  if constexpr (BF16) return fabsf(v) <= 3.0e38f;
+  return fabsf(v) < 2147483648.0f;
+}
+
+// The four 16-bit pieces of v, packed [b0 | b1], [b2 | b3].  Each piece is
+// the 16-bit rounding of the remainder scaled by 1 / weight; an fp16 piece
+// that would be subnormal is set to 0 and its value left to the pieces below,
+// so the result never depends on how the tensor core treats subnormals.  The
+// remainder updates are exact (Sterbenz: the subtracted value is within a
+// factor 2 of the remainder).
+template <bool BF16>
+__device__ __forceinline__ uint2 ext_pieces(float v) {
+  float b[4];
+  float r = v;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (BF16 && i == 3) {
+      b[i] = 0.f;
+      continue;
+    }
+    float x = unpack2<BF16>(pack2<BF16>(r * ext_inv_weight<BF16>(i), 0.f)).x;
+    if (!BF16 && fabsf(x) < 6.103515625e-05f) x = 0.f;
+    b[i] = x;
+    r -= x * ext_weight<BF16>(i);
+  }
+  return make_uint2(pack2<BF16>(b[0], b[1]), pack2<BF16>(b[2], b[3]));
 }
 
 template <bool BF16>
@@ -277,12 +329,14 @@ __global__ void __launch_bounds__(512, 1)
     tmem_relinquish();
   }
   if (warp == 3) {
-    // A_ext: [sel_s: rows of 1,1,0,..] [zeros] [sel_d: rows of 0,0,1,1,0,..] [zeros]
-    const uint32_t one = BF16 ? 0x3F80u : 0x3C00u;
+    // A_ext: [sel_s: rows of w0,w1,w2,w3,0,..] [zeros] [sel_d: rows of 0,0,0,0,w0,w1,w2,w3] [zeros]
+    // (the piece weights of ext_pieces).
     uint32_t* a = reinterpret_cast<uint32_t*>(smem + L::kAExtOff);
     for (int i = lane; i < L::kAExtBytes / 4; i += 32) {
       const int cm = i / 32, w = i % 4;  // core matrix, 32-bit word within a 16-byte row
-      a[i] = (cm == 0 && w == 0) || (cm == 2 && w == 1) ? (one | (one << 16)) : 0u;
+      const bool sel = (cm == 0 && w < 2) || (cm == 2 && w >= 2);
+      const int p = 2 * (w & 1);          // first piece of this word
+      a[i] = sel ? pack2<BF16>(ext_weight<BF16>(p), ext_weight<BF16>(p + 1)) : 0u;
     }
     fence_proxy_async_smem();
   }
@@ -439,15 +493,15 @@ __global__ void __launch_bounds__(512, 1)
     mbar_drain(mma_done, 0);
   } else if (warp == 3) {
     // ------------------------------------------------------------ B_ext writer
-    // Row q of B_ext: [s_hi, s_lo, d_hi, d_lo, 0, 0, 0, 0] with s = -LSE_q /
-    // scale (-log2(e) LSE_q when scale == 0) and d = -D_q, each split into a
-    // 16-bit value and the 16-bit rounding of its remainder.
+    // Row q of B_ext: [s0, s1, s2, s3, d0, d1, d2, d3], the 16-bit pieces
+    // (ext_pieces) of s = -LSE_q / scale (-log2(e) LSE_q when scale == 0)
+    // and d = -D_q.  A term outside the pieces' range (fp16: |LSE_q / scale|
+    // or |D_q| >= 2^31) is recorded as ATTN_ERR_RANGE in the device status
+    // word; its pieces are then zero rather than infinite, so the products
+    // stay finite.
     const float inv_c = scale == 0.f ? 1.f : 1.f / scale_log2;  // nlse2 = -log2(e) LSE
     uint4* bext = reinterpret_cast<uint4*>(smem + L::kBExtOff);
-    auto split = [](float v) {
-      const float hi = unpack2<BF16>(pack2<BF16>(v, 0.f)).x;
-      return pack2<BF16>(hi, v - hi);
-    };
+    bool range_ok = true;
     for (int it = 0; it < n_it; ++it) {
       const size_t vbase = qslab + static_cast<size_t>(i0 + it) * kBwdTile;
       const int q_valid = nq - (i0 + it) * kBwdTile;
@@ -457,13 +511,22 @@ __global__ void __launch_bounds__(512, 1)
         const bool in = lane + 32 * k < q_valid;  // rows past the sequence: zeros (their P is masked)
         sv[k] = in ? nlse2[vbase + lane + 32 * k] * inv_c : 0.f;
         dv4[k] = in ? -dvec[vbase + lane + 32 * k] : 0.f;
+        if (!ext_in_range<BF16>(sv[k]) || !ext_in_range<BF16>(dv4[k])) {
+          range_ok = false;
+          sv[k] = ext_in_range<BF16>(sv[k]) ? sv[k] : 0.f;
+          dv4[k] = ext_in_range<BF16>(dv4[k]) ? dv4[k] : 0.f;
+        }
       }
       if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(bext_free, (it - 1) & 1, abort_flag))) break;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) bext[lane + 32 * k] = make_uint4(split(sv[k]), split(dv4[k]), 0u, 0u);
+      for (int k = 0; k < 4; ++k) {
+        const uint2 s4 = ext_pieces<BF16>(sv[k]), d4 = ext_pieces<BF16>(dv4[k]);
+        bext[lane + 32 * k] = make_uint4(s4.x, s4.y, d4.x, d4.y);
+      }
       fence_proxy_async_smem();
       mbar_arrive(bext_full);
     }
+    if (!__all_sync(0xffffffffu, range_ok) && lane == 0) atomicExch(&g_device_status, kStatusRange);
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ P and dS
     const int h = (warp - 4) >> 2;  // query columns [64h, 64h + 64)

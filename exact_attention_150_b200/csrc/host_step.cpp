@@ -68,6 +68,12 @@ bool make_plan(int B, int H, int Nq, int Nk, int d, int chunks, Plan* p) {
   p->chunks = static_cast<int>(p->bh < chunks ? p->bh : chunks);
   p->per_chunk = (p->bh + p->chunks - 1) / p->chunks;
   p->chunks = static_cast<int>((p->bh + p->per_chunk - 1) / p->per_chunk);  // no empty chunk
+  // Each chunk is one attn_fwd / attn_bwd call with B = 1, H = per_chunk: it
+  // must meet their shape rules (tile counts, grid size), checked here so
+  // that a shape they would refuse is refused before any copy is enqueued.
+  const long long tq = (Nq + 127) / 128, tk = (Nk + 127) / 128;
+  if (tq > 65535 || tk > 65535 || p->per_chunk * tq > 0x7fffffffLL || p->per_chunk * tk > 0x7fffffffLL)
+    return false;
   const size_t qbytes = static_cast<size_t>(p->bh) * Nq * d * p->eb;
   const size_t kbytes = static_cast<size_t>(p->bh) * Nk * d * p->eb;
   size_t at = 0;

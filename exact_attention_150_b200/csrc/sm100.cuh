@@ -18,6 +18,7 @@ namespace attn {
 // Status codes mirrored from attn.h (kept numeric to avoid a header cycle).
 constexpr int kStatusTimeout = 4;
 constexpr int kStatusSmem = 6;
+constexpr int kStatusRange = 7;
 
 // Device status word: 0 = OK, otherwise an attn_status code.
 __device__ int g_device_status;

@@ -19,7 +19,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libattn.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "attn.h")
 
-ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_SCRATCH_LIMIT, ATTN_ERR_SMEM = range(7)
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_SCRATCH_LIMIT, ATTN_ERR_SMEM, \
+    ATTN_ERR_RANGE = range(8)
 ATTN_FP16, ATTN_BF16 = 0, 1
 ATTN_BWD_ALL, ATTN_BWD_PREPROCESS, ATTN_BWD_MAIN, ATTN_BWD_CONVERT = range(4)
 ATTN_CAUSAL_NONE, ATTN_CAUSAL_TOP_LEFT, ATTN_CAUSAL_BOTTOM_RIGHT = range(3)

@@ -62,7 +62,9 @@
  *   that exceeds its time limit makes the kernel record ATTN_ERR_TIMEOUT in a
  *   device status word and return early, and a kernel that finds less shared
  *   memory than its tiles need records ATTN_ERR_SMEM and returns without
- *   work; attn_last_device_status() reads the word.
+ *   work; attn_last_device_status() reads the word.  An fp16 backward whose
+ *   per-query terms leave the range the kernel can represent records
+ *   ATTN_ERR_RANGE there (see attn_bwd).
  */
 #ifndef ATTN_H_
 #define ATTN_H_
@@ -80,7 +82,8 @@ typedef enum {
   ATTN_ERR_CUDA = 3,
   ATTN_ERR_TIMEOUT = 4,
   ATTN_ERR_SCRATCH_LIMIT = 5,
-  ATTN_ERR_SMEM = 6
+  ATTN_ERR_SMEM = 6,
+  ATTN_ERR_RANGE = 7
 } attn_status;
 
 typedef enum { ATTN_FP16 = 0, ATTN_BF16 = 1 } attn_dtype;
@@ -166,6 +169,15 @@ size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d);
  *                unspecified.  It must not be shared by calls that overlap.
  * dQ is accumulated with fp32 atomic additions, so its last bits may differ
  * between runs; dK and dV are deterministic.
+ * Any finite scale is accepted, 0 and negative ones included.  The kernel
+ * adds the per-query terms -LSE_i / scale and -D_i to its fp32 products as
+ * pieces of the 16-bit input type; in fp16 they are exact for
+ * |LSE_i / scale| < 2^31 and |D_i| < 2^31 (for example any |scale| >= 1e-8
+ * with |LSE| <= 20).  Beyond that the call records ATTN_ERR_RANGE in the
+ * device status word (attn_last_device_status) and its gradients are not
+ * meaningful.  bf16 has no such limit.  As in every 16-bit attention
+ * backward, dS = P * (dP - D) is rounded to the input type before its two
+ * products, so |dP - D| beyond the type's range overflows there.
  */
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
@@ -334,7 +346,9 @@ attn_status attn_selftest_wait_timeout(int limit_us, int* result, void* stream);
 /*
  * Synchronises `stream`, then returns and clears the device status word that
  * kernels of this library set when a bounded wait times out
- * (ATTN_ERR_TIMEOUT), or ATTN_ERR_CUDA if the synchronisation itself fails.
+ * (ATTN_ERR_TIMEOUT), when shared memory is short (ATTN_ERR_SMEM) or when an
+ * fp16 backward's per-query terms are out of range (ATTN_ERR_RANGE), or
+ * ATTN_ERR_CUDA if the synchronisation itself fails.
  * ATTN_OK means no kernel of this library has recorded an error since the
  * previous call on this device.
  */

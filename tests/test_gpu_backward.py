@@ -154,10 +154,31 @@ def test_long_context_workload_windows_and_identities():
                                           q_offset=n - win)
             parity.assert_grad(parity.f64(dkf[s, n - win:]), rdk[n - win:], "dK keys>=N-1024", tag)
             parity.assert_grad(parity.f64(dvf[s, n - win:]), rdv[n - win:], "dV keys>=N-1024", tag)
+        if s in (6, 13):
+            _check_interior_key_tile(qf[s], kf[s], vf[s], dof[s], dkf[s], dvf[s], w.scale, 64, tag)
         # Whole run: sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i.
         gk, gv, gdo = parity.f64(dkf[s]), parity.f64(dvf[s]), parity.f64(dof[s])
         assert np.linalg.norm(gk.sum(0)) <= parity.GRAD_TOL * np.linalg.norm(gk), tag + " sum dK"
         assert np.linalg.norm(gv.sum(0) - gdo.sum(0)) <= parity.GRAD_TOL * np.linalg.norm(gv), tag + " sum dV"
+
+
+def _check_interior_key_tile(q, k, v, do, dk, dv, scale, tile, tag, chunk=512):
+    """dK and dV of key tile `tile` (keys [128 t, 128 t + 128)) of one causal
+    head against the exact oracle.  Those keys receive gradient from query
+    rows i >= 128 t; each chunk of such rows sees only keys [0, chunk end), so
+    the oracle runs on that prefix and its dK, dV contributions are summed."""
+    n = q.shape[0]
+    k0, k1 = 128 * tile, 128 * tile + 128
+    rdk = np.zeros((128, q.shape[1]))
+    rdv = np.zeros((128, q.shape[1]))
+    for r0 in range(k0, n, chunk):
+        r1 = min(r0 + chunk, n)
+        _, ck, cv = oracle.backward(parity.f64(q[r0:r1]), parity.f64(k[:r1]), parity.f64(v[:r1]),
+                                    parity.f64(do[r0:r1]), scale, True, q_offset=r0)
+        rdk += ck[k0:k1]
+        rdv += cv[k0:k1]
+    parity.assert_grad(parity.f64(dk[k0:k1]), rdk, f"dK key tile {tile}", tag)
+    parity.assert_grad(parity.f64(dv[k0:k1]), rdv, f"dV key tile {tile}", tag)
 
 
 # ------------------------------------------------------- deterministic mode
@@ -201,3 +222,80 @@ def test_deterministic_backward_is_bit_reproducible(causal):
     ref = run_bwd_det(q, k, v, do, causal, 1 / math.sqrt(128), False)
     for a, b in zip(runs[0], ref):
         assert parity.rel_fro(parity.f64(a), parity.f64(b)) < 1e-2
+
+
+# ------------------------------------------------- fp16 range of the row terms
+#
+# The backward adds -LSE_i / scale and -D_i to its fp32 products as 16-bit
+# pieces.  In fp16 a single piece overflows past 65504; these cases all have
+# terms beyond that and must still match the oracle.
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal,nq,nk", [(True, 777, 777), ("bottom_right", 300, 900)])
+@pytest.mark.parametrize("scale", [1e-4, 1e-5, -1e-4])
+def test_backward_fp16_small_scale(scale, causal, nq, nk, d):
+    """|LSE / scale| ~ ln(keys) / |scale| reaches 6.9e4 .. 6.9e5 here."""
+    q, k, v, do = draw(1, 2, nq, nk, d, torch.float16, seed=81 + nq + d, with_grad=True)
+    check_grads_all_slices(q, k, v, do, causal, scale, f"fp16 scale {scale} d{d} Nq{nq} Nk{nk} causal={causal}")
+
+
+def _mean_free(x):
+    return x - x.mean(-1, keepdim=True)
+
+
+def test_backward_fp16_large_scores():
+    """Every score q.k is about 24^2 * 128 = 73728 (a common offset plus a
+    spread of about 11), so LSE / scale is past fp16's 65504 on every row
+    while the softmax stays spread out.  LSE itself is about 6.5e3 here, and
+    the fp32 sums of scores that large round at about 2^-24 |q.k| scale per
+    step, a few 1e-3 in all: LSE is held to a relative 1e-6 instead of the
+    absolute 1e-3 that N(0,1) inputs get.  O and the gradients keep their
+    bars."""
+    g = torch.Generator().manual_seed(83)
+    n, d = 384, 128
+    scale = 1 / math.sqrt(d)
+    q = (24.0 + _mean_free(torch.randn(1, 2, n, d, generator=g))).half()
+    k = (24.0 + _mean_free(torch.randn(1, 2, n, d, generator=g))).half()
+    v = torch.randn(1, 2, n, d, generator=g).half()
+    do = torch.randn(1, 2, n, d, generator=g).half()
+    o, lse, dq, dk, dv = run_fwd_bwd(q, k, v, do, True, scale)
+    for s in range(2):
+        args = [parity.f64(t[0, s]) for t in (q, k, v, do)]
+        ro, rlse, _ = oracle.forward(*args[:3], scale, True)
+        rdq, rdk, rdv = oracle.backward(*args, scale, True)
+        tag = f"fp16 large scores slice {s}"
+        assert np.max(np.abs(rlse)) > 6000 and np.max(np.abs(rlse / scale)) > 65504
+        parity.assert_o(parity.f64(o[0, s]), ro, q.dtype, tag)
+        rel = np.max(np.abs(parity.f64(lse[0, s]) - rlse) / np.abs(rlse))
+        assert rel <= 1e-6, f"{tag}: LSE relative error {rel:.3e}"
+        parity.assert_grad(parity.f64(dq[0, s]), rdq, "dQ", tag)
+        parity.assert_grad(parity.f64(dk[0, s]), rdk, "dK", tag)
+        parity.assert_grad(parity.f64(dv[0, s]), rdv, "dV", tag)
+
+
+def test_backward_fp16_large_row_term_d():
+    """V = 2 + N(0,1) and dO ~ 4000 N(0,1): D_i = dO_i . O_i is about
+    2 sum_c dO_ic, past fp16's range on most rows, while dP - D stays near
+    4e4 and dS = P (dP - D) well inside it."""
+    g = torch.Generator().manual_seed(85)
+    n, d = 512, 128
+    q = torch.randn(1, 2, n, d, generator=g).half()
+    k = torch.randn(1, 2, n, d, generator=g).half()
+    v = (2.0 + torch.randn(1, 2, n, d, generator=g)).half()
+    do = (4000.0 * torch.randn(1, 2, n, d, generator=g)).half()
+    dvec = (parity.f64(do) * 2.0).sum(-1)
+    assert np.mean(np.abs(dvec) > 65504) > 0.3  # the case this test is about
+    check_grads_all_slices(q, k, v, do, False, 1 / math.sqrt(d), "fp16 large D")
+
+
+def test_backward_fp16_out_of_range_term_is_reported():
+    """scale = 1e-9: |LSE / scale| ~ 5e9 is beyond what the fp16 pieces hold
+    (2^31); the kernel records ATTN_ERR_RANGE instead of returning NaN
+    silently, and the context stays usable."""
+    q, k, v, do = draw(1, 2, 256, 256, 64, torch.float16, seed=87, with_grad=True)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = native.forward(qd, kd, vd, causal=True, scale=1e-9)
+    native.backward(qd, kd, vd, o, lse, dod, causal=True, scale=1e-9)
+    assert native.attn_last_device_status() == native.ATTN_ERR_RANGE
+    assert native.attn_last_device_status() == native.ATTN_OK  # read clears it
+    check_grads_all_slices(q, k, v, do, True, 1e-4, "after a range error")

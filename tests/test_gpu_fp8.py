@@ -1,7 +1,7 @@
 """FP8 forward parity: attn_fwd_fp8 (through the C ABI) against the fp64
 oracle's exact attention of the descaled E4M3 inputs, with the E4M3
 tolerances of tests/parity.py: one 128 x 128 tile per problem under each
-mask, and constant V.  tests/pending_gpu_fp8.py holds the wider cases.
+mask, and constant V.  tests/test_gpu_fp8_wide.py holds the wider cases.
 """
 
 import math

@@ -1,10 +1,7 @@
 """Wider FP8 forward parity cases: shapes spanning several tiles, ragged
 tails, Nq != Nk under each mask, other descale factors and scales, sampled
-rows of the long-context FP8 shape, and empty or invalid calls.
-
-This module's name keeps it out of pytest's default collection, so that
-``pytest tests -m gpu`` does not run it; run it by name on a B200:
-``python -m pytest tests/pending_gpu_fp8.py -q``.
+rows of the long-context FP8 shape, empty or invalid calls, and the packed
+variable-length form (attn_fwd_fp8_varlen).
 """
 
 import math

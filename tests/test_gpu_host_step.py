@@ -5,10 +5,6 @@ With the deterministic backward on both sides every output must agree bit
 for bit: each chunk runs the same kernels on the same slices.  Cases cover
 chunk counts that do not divide B*H, an odd Nq (each chunk's LSE block has
 its own alignment), B > 1, both dtypes and the masks.
-
-This module's name keeps it out of pytest's default collection, so that
-``pytest tests -m gpu`` does not run it; run it by name on a B200:
-``python -m pytest tests/pending_gpu_host_step.py -q``.
 """
 
 import math
