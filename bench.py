@@ -374,7 +374,7 @@ def run_ours(args):
         if ev is not None:
             ev[1].record(stream)
         if args.deterministic:
-            # One call: order counters, preprocess, main and convert kernels.
+            # One call: preprocess, dK/dV and dQ kernels.
             bwd(native.ATTN_BWD_ALL)
             if ev is not None:
                 for e in ev[2:]:
@@ -390,7 +390,7 @@ def run_ours(args):
         if ev is not None:
             ev[4].record(stream)
 
-    launches_per_step = (5 if args.deterministic else 4) if w.backward else 1
+    launches_per_step = 4 if w.backward else 1
     for _ in range(max(args.warmup, 0)):
         step()
     torch.cuda.synchronize(device)
@@ -424,7 +424,7 @@ def run_ours(args):
     kernels = {"fwd_kernel": {"ms": fwd_ms, "tflops": w.fwd_flops() / fwd_ms / 1e9, "gbs": fwd_bytes / fwd_ms / 1e6}}
     if w.backward and args.deterministic:
         det_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-        kernels["bwd_deterministic (order counters + 3 kernels)"] = {"ms": det_ms,
+        kernels["bwd_deterministic (preprocess, dK/dV and dQ kernels)"] = {"ms": det_ms,
                                                                       "tflops": w.bwd_flops() / det_ms / 1e9}
         dom_name, dom_ms, dom_flops = "bwd_deterministic", det_ms, w.bwd_flops()
     elif w.backward:
@@ -438,7 +438,7 @@ def run_ours(args):
         dom_name, dom_ms, dom_flops = "bwd_main_kernel", main_ms, w.bwd_flops()
     else:
         dom_name, dom_ms, dom_flops = "fwd_kernel", fwd_ms, w.fwd_flops()
-    spans = {"fwd_kernel": (0, 1), "bwd_deterministic (order counters + 3 kernels)": (1, 2),
+    spans = {"fwd_kernel": (0, 1), "bwd_deterministic (preprocess, dK/dV and dQ kernels)": (1, 2),
              "bwd_pre_kernel": (1, 2), "bwd_main_kernel": (2, 3), "bwd_post_kernel": (3, 4)}
     add_spread(kernels, evs, spans)
     for name, kinfo in kernels.items():

@@ -11,6 +11,7 @@
 #include <utility>
 
 #include "attn.h"
+#include "bwd_dq_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "fwd_kernel.cuh"
 #include "trace.h"
@@ -179,8 +180,8 @@ Problem varlen_problem(int B, int H, int total_q, int total_k, int max_q, int ma
 
 // Backward workspace of a problem, in 4-byte words: dQ accumulator
 // [(rows + pad) * d] | D [rows] | -log2(e) LSE [rows] | (16-byte aligned)
-// order counters [problems][qtiles] of the deterministic backward, with
-// rows = slabs * rows_q.  The pad takes the reductions of the ragged last
+// [problems][qtiles] words that no kernel uses at present (they keep the
+// size attn_bwd_workspace_bytes documents), with rows = slabs * rows_q.  The pad takes the reductions of the ragged last
 // query tile's masked rows (exact zeros; see pad_rows); in a packed batch
 // any sequence's last tile can reach up to 127 rows past the total.
 struct WsLayout {
@@ -214,6 +215,11 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// The backward kernels of one call.  DET = false: preprocess (which also
+// zeroes the fp32 dQ accumulator), the main kernel with atomic dQ
+// reductions, and the dQ convert.  DET = true: preprocess, the main kernel
+// for dK and dV only, and the dQ kernel, which owns its dQ rows and writes
+// them directly (no accumulator, no atomics, the same bits on every run).
 template <int D, bool BF16, bool CAUSAL, bool DET>
 attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                        const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv, float* ws,
@@ -224,35 +230,41 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   float* dqacc = ws;
   float* dvec = ws + w.dvec;
   float* nlse2 = ws + w.nlse2;
-  int* dq_order = DET ? reinterpret_cast<int*>(ws + w.counters) : nullptr;
+  const float scale_log2 = scale * 1.4426950408889634f;
 
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_PREPROCESS) {
-    if (DET && cudaMemsetAsync(dq_order, 0, static_cast<size_t>(w.ncounters) * sizeof(int), st) != cudaSuccess)
-      return ATTN_ERR_CUDA;
     constexpr int kRowsPerBlock = 256 / (D / 8);
     const long long pre_blocks = (qrows + kRowsPerBlock - 1) / kRowsPerBlock;
     attn::bwd_pre_kernel<D, BF16><<<static_cast<unsigned>(pre_blocks), 256, 0, st>>>(
-        static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, dvec, nlse2, dqacc, qrows);
+        static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, dvec, nlse2, DET ? nullptr : dqacc,
+        qrows);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_MAIN) {
-    auto kern = attn::bwd_main_kernel<D, BF16, CAUSAL, DET>;
+    auto kern = attn::bwd_main_kernel<D, BF16, CAUSAL, !DET>;
     if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
     // Every CTA of a problem streams its Q and dO rows, their LSE and D, and
-    // adds into its dQ accumulator rows.  The deterministic mode keeps
-    // problem-fastest order: its key tiles take turns on each query tile, and
-    // a problem whose key tiles were all resident at once would leave key
-    // tile j waiting about 2j steps.
-    const int group =
-        DET ? pb.problems : attn::order_group((8.0 * D + 8.0) * avg_rows(pb.rows_q, pb), pb.problems);
+    // (atomic dQ) adds into its dQ accumulator rows.
+    const int group = attn::order_group((8.0 * D + 8.0) * avg_rows(pb.rows_q, pb), pb.problems);
     const unsigned grid = static_cast<unsigned>(pb.problems) * static_cast<unsigned>(pb.ktiles);
     kern<<<grid, 512, L::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, dqacc, static_cast<uint16_t*>(dk),
-                                       static_cast<uint16_t*>(dv), dq_order, pb.cu_q, pb.cu_k, pb.H, pb.rows_q,
-                                       pb.rows_k, pb.bottom_right, pb.qtiles, scale, scale * 1.4426950408889634f,
-                                       pb.problems, pb.ktiles, group);
+                                       static_cast<uint16_t*>(dv), pb.cu_q, pb.cu_k, pb.H, pb.rows_q, pb.rows_k,
+                                       pb.bottom_right, pb.qtiles, scale, scale_log2, pb.problems, pb.ktiles, group);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    if constexpr (DET) {
+      using LQ = attn::BwdDqLayout<D>;
+      auto kq = attn::bwd_dq_kernel<D, BF16, CAUSAL>;
+      if (set_smem(kq, LQ::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
+      // Every CTA of a problem streams its K and V.
+      const int gq = attn::order_group(4.0 * D * avg_rows(pb.rows_k, pb), pb.problems);
+      const unsigned gridq = static_cast<unsigned>(pb.problems) * static_cast<unsigned>(pb.qtiles);
+      kq<<<gridq, 384, LQ::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, static_cast<uint16_t*>(dq), pb.cu_q, pb.cu_k,
+                                         pb.H, pb.rows_q, pb.rows_k, pb.bottom_right, scale, scale_log2, pb.problems,
+                                         pb.qtiles, gq);
+      if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    }
   }
-  if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_CONVERT) {
+  if (!DET && (phase == ATTN_BWD_ALL || phase == ATTN_BWD_CONVERT)) {
     const long long n8 = qrows * D / 8;
     long long post_blocks = (n8 + 255) / 256;
     if (post_blocks > 148LL * 16) post_blocks = 148LL * 16;

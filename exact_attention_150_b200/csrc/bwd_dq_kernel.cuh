@@ -1,0 +1,398 @@
+// bwd_dq_kernel.cuh -- dQ of the attention backward, one query tile per CTA.
+//
+// The backward pass recomputes the attention probabilities from Q, K and the
+// saved row log-sum-exp instead of storing them (page "FlashAttention 核心原理",
+// part 2 item 3).  bwd_main_kernel does so per key tile and accumulates dK and
+// dV; this kernel does so per query tile and accumulates
+//   dQ_i = scale * sum_j dS_ij K_j,   dS = P * (dO V^T - D),
+//   P = exp(scale * Q K^T - LSE)
+// over the key tiles j that the query tile sees.  Each CTA owns its dQ rows,
+// so dQ needs no atomic additions and comes out the same, bit for bit, on
+// every run; together with bwd_main_kernel<..., DQ = false> it is the
+// reproducible backward.
+//
+// CTA layout (384 threads, one CTA per SM):
+//   warp 0       TMA producer: Q_i and dO_i once, then K_0, V_0, K_1, V_1, ...
+//                through a ring of shared-memory slots
+//   warp 1       MMA issuer (one elected lane per group)
+//   warp 2       tensor-memory allocation / release
+//   warp 3       idle
+//   warps 4-7    P and dS for key columns [0, 64) of every key tile
+//   warps 8-11   P and dS for key columns [64, 128)
+//                (thread = query row = TMEM lane: a row's LSE and D are
+//                per-thread values; each warpgroup also writes half of the
+//                head dimension of dQ at the end)
+// Tensor memory (512 columns):
+//   [0, 128), [128, 256)  S of even / odd key tiles (fp32); dS of the tile is
+//                         written in place, 16-bit packed, keys [64h, 64h+64)
+//                         in columns [64h, 64h+32)
+//   [256, 384)            dP = dO V^T (fp32)
+//   [384, 384+D)          dQ accumulator (fp32)
+// Products per key tile j: S(j) = Q K_j^T and dP(j) = dO V_j^T with both
+// operands in shared memory, dQ += dS(j) K_j with dS from tensor memory.
+// Issue order: S(0), dP(0), S(1), then per j: dP(j+1) once the softmax warps
+// have read dP(j), dQ(j) once they have written dS(j), S(j+2) into the
+// buffer that dQ(j) has just read.  The softmax warps therefore always find
+// the next S and dP ready when they finish a tile.
+#pragma once
+
+#include "sm100.cuh"
+#include "tile_order.h"
+
+namespace attn {
+
+template <int D>
+struct BwdDqLayout {
+  static constexpr int kTileRows = 128;
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kChunks = kRowBytes / 128;      // 128-byte column chunks per row
+  static constexpr int kChunkBytes = kTileRows * 128;  // one 128-row chunk
+  static constexpr int kTileBytes = kTileRows * kRowBytes;
+  static constexpr int kSlots = D == 128 ? 5 : 10;     // K/V ring slots
+  static constexpr int kQOff = 0;
+  static constexpr int kDOOff = kQOff + kTileBytes;
+  static constexpr int kRingOff = kDOOff + kTileBytes;
+  static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+  // qd_full, kv_full[kSlots], kv_empty[kSlots], s_full[2], dp_full, dp_read,
+  // ds_full, dq_done, mma_done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 7;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024 <= 232448 ? kBytes + 1024 : 232448;
+  static_assert(kBytes <= 232448, "shared memory budget");
+  static constexpr uint32_t kColS = 0;     // S buffer b at kColS + 128 b
+  static constexpr uint32_t kColDP = 256;
+  static constexpr uint32_t kColDQ = 384;
+  static_assert(kColDQ + D <= 512, "tensor memory budget");
+};
+
+// dvec and nlse2 hold D_i and -log2(e) LSE_i per query row of the tensor
+// maps' slabs (bwd_pre_kernel); dq_ptr is the 16-bit dQ.  The grid is the
+// query tiles of every problem in the grouped launch order of tile_order.h.
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const float* __restrict__ dvec, const float* __restrict__ nlse2, uint16_t* __restrict__ dq_ptr,
+                  const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H, int Nq, int Nk,
+                  int bottom_right, float scale, float scale_log2, int problems, int grid_tiles, int group) {
+  using L = BwdDqLayout<D>;
+  constexpr int kT = L::kTileRows;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* qd_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + L::kSlots;
+  uint64_t* s_full = kv_empty + L::kSlots;  // [2], by key-tile parity
+  uint64_t* dp_full = s_full + 2;
+  uint64_t* dp_read = dp_full + 1;          // 256 arrivals: dP loaded by the softmax warps
+  uint64_t* ds_full = dp_read + 1;          // 256 arrivals: dS written
+  uint64_t* dq_done = ds_full + 1;
+  uint64_t* mma_done = dq_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  // The problem of this CTA (as in the forward): slab z, rows [q0, q0 + nq)
+  // of the queries and [k0, k0 + nk) of the keys, offsets of a packed batch
+  // clamped to the slab.
+  int px, ty;
+  grouped_order(blockIdx.x, problems, grid_tiles, group, &px, &ty);
+  int z = px, q0 = 0, k0 = 0, nq = Nq, nk = Nk;
+  if (cu_q != nullptr) {
+    const int b = px / H;
+    z = px - b * H;
+    auto clamp = [](int v, int hi) { return v < 0 ? 0 : (v > hi ? hi : v); };
+    q0 = clamp(cu_q[b], Nq);
+    k0 = clamp(cu_k[b], Nk);
+    nq = clamp(cu_q[b + 1], Nq) - q0;
+    nk = clamp(cu_k[b + 1], Nk) - k0;
+    nq = nq < 0 ? 0 : nq;
+    nk = nk < 0 ? 0 : nk;
+  }
+  const int nqt = (nq + kT - 1) / kT;
+  const int nkt = (nk + kT - 1) / kT;
+  if (ty >= nqt) return;  // a sequence shorter than the grid
+  // Causal: the heaviest query tiles are launched first.
+  const int qt = CAUSAL ? (nqt - 1 - ty) : ty;
+  // Key tiles this query tile sees (causal: query i sees key k iff
+  // k <= i + off, off = 0 top-left, nk - nq bottom-right).
+  const int off = bottom_right ? nk - nq : 0;
+  int n = nkt;
+  if (CAUSAL) {
+    const int last_row = qt * kT + kT - 1 < nq - 1 ? qt * kT + kT - 1 : nq - 1;
+    const int last_key = last_row + off < nk - 1 ? last_row + off : nk - 1;
+    n = last_key < 0 ? 0 : last_key / kT + 1;
+  }
+  const size_t grow0 = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kT;  // first row of the tile
+  if (n == 0) {
+    // No row of this tile sees a key: its softmax is empty and dQ = 0.
+    const int rows = nq - qt * kT < kT ? nq - qt * kT : kT;
+    for (int e = threadIdx.x; e < rows * D / 8; e += blockDim.x)
+      reinterpret_cast<uint4*>(dq_ptr + grow0 * D)[e] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+
+  // Refuse to run (and report) if alignment left too little shared memory.
+  if (static_cast<uint32_t>(smem - smem_raw) + L::kBytes > dynamic_smem_bytes()) {
+    if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusSmem);
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(qd_full, 1);
+    for (int i = 0; i < L::kSlots; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(dp_full, 1);
+    mbar_init(dp_read, 256);
+    mbar_init(ds_full, 256);
+    mbar_init(dq_done, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Ring items: K_j is item 2j, V_j item 2j + 1 (j < n).
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(qd_full, 2 * L::kTileBytes);
+      for (int c = 0; c < L::kChunks; ++c) {
+        tma_load_3d(smem + L::kQOff + c * L::kChunkBytes, &tm_q, qd_full, c * 64, q0 + qt * kT, z);
+        tma_load_3d(smem + L::kDOOff + c * L::kChunkBytes, &tm_do, qd_full, c * 64, q0 + qt * kT, z);
+      }
+      int item = 0;
+      bool ok = true;
+      for (; ok && item < 2 * n; ++item) {
+        const int slot = item % L::kSlots;
+        if (!mbar_wait(&kv_empty[slot], ((item / L::kSlots) & 1) ^ 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
+        uint8_t* dst = smem + L::kRingOff + slot * L::kTileBytes;
+        const CUtensorMap* map = (item & 1) ? &tm_v : &tm_k;
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * 64, k0 + (item >> 1) * kT, z);
+      }
+      if (!ok) {
+        // Let the copies already issued land before the CTA exits.
+        mbar_drain(qd_full, 0);
+        const int first = item > L::kSlots ? item - L::kSlots : 0;
+        for (int i = first; i < item; ++i) mbar_drain(&kv_full[i % L::kSlots], (i / L::kSlots) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // K-major x K-major
+    constexpr uint32_t kIdQ = idesc_f16(BF16, 128, D, false, true);     // dS (TMEM) x K MN-major
+    const uint32_t ring_base = smem_u32(smem + L::kRingOff);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    auto slot_addr = [&](int item) { return ring_base + (item % L::kSlots) * L::kTileBytes; };
+    auto wait_item = [&](int item) { return wait_all(&kv_full[item % L::kSlots], (item / L::kSlots) & 1); };
+    const uint64_t qd = sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+    const uint64_t dod = sdesc_sw128(smem_u32(smem + L::kDOOff), 16, 1024);
+    // A K-major SW128 operand steps 32 bytes per K step of 16 inside a
+    // 128-byte row, and one 16 KB chunk per 64 columns.
+    auto kstep = [](int ks) { return static_cast<uint64_t>(((ks >> 2) * L::kChunkBytes + (ks & 3) * 32) >> 4); };
+    auto issue_s = [&](int j) {  // S(j) = Q K_j^T into buffer j & 1
+      const uint64_t kd = sdesc_sw128(slot_addr(2 * j), 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        mma_ss(tmem + L::kColS + 128 * (j & 1), qd + kstep(ks), kd + kstep(ks), kIdS, ks > 0 ? 1u : 0u);
+    };
+    auto issue_dp = [&](int j) {  // dP(j) = dO V_j^T
+      const uint64_t vd = sdesc_sw128(slot_addr(2 * j + 1), 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        mma_ss(tmem + L::kColDP, dod + kstep(ks), vd + kstep(ks), kIdS, ks > 0 ? 1u : 0u);
+    };
+    // dQ += dS(j) K_j: A = dS from buffer j & 1 (key step ks of 16 keys:
+    // keys [64h, 64h + 64) sit in columns [64h, 64h + 32), 8 per step),
+    // B = K_j MN-major (16 key rows of 128 bytes per step).
+    auto issue_dq = [&](int j) {
+      const uint64_t kmn = sdesc_sw128(slot_addr(2 * j), L::kChunkBytes, 1024);
+#pragma unroll
+      for (int ks = 0; ks < kT / 16; ++ks) {
+        const uint32_t ds_col = tmem + L::kColS + 128 * (j & 1) + 64 * (ks >> 2) + 8 * (ks & 3);
+        mma_ts(tmem + L::kColDQ, ds_col, kmn + 128 * ks, kIdQ, (j > 0 || ks > 0) ? 1u : 0u);
+      }
+    };
+    bool ok = wait_all(qd_full, 0) && wait_item(0) && wait_item(1);
+    if (ok) {
+      tc_fence_after();
+      if (elect_one()) {
+        issue_s(0);
+        mma_commit(&s_full[0]);
+        issue_dp(0);
+        mma_commit(dp_full);
+        mma_commit(&kv_empty[1 % L::kSlots]);  // V_0 read
+      }
+      __syncwarp();
+    }
+    if (ok && n > 1 && (ok = wait_item(2))) {
+      tc_fence_after();
+      if (elect_one()) {
+        issue_s(1);
+        mma_commit(&s_full[1]);
+      }
+      __syncwarp();
+    }
+    for (int j = 0; ok && j < n; ++j) {
+      if (j + 1 < n) {
+        // dP(j+1) overwrites dP(j): the softmax warps have loaded it.
+        if (!(ok = wait_all(dp_read, j & 1))) break;
+        if (!(ok = wait_item(2 * j + 3))) break;
+        tc_fence_after();
+        if (elect_one()) {
+          issue_dp(j + 1);
+          mma_commit(dp_full);
+          mma_commit(&kv_empty[(2 * j + 3) % L::kSlots]);  // V_{j+1} read
+        }
+        __syncwarp();
+      }
+      if (!(ok = wait_all(ds_full, j & 1))) break;
+      tc_fence_after();
+      if (elect_one()) {
+        issue_dq(j);
+        mma_commit(&kv_empty[(2 * j) % L::kSlots]);  // K_j read by S(j) and dQ(j)
+        if (j == n - 1) mma_commit(dq_done);
+      }
+      __syncwarp();
+      if (j + 2 < n) {
+        if (!(ok = wait_item(2 * j + 4))) break;
+        tc_fence_after();
+        if (elect_one()) {
+          issue_s(j + 2);  // into the buffer whose dS dQ(j) (issued above) consumes first
+          mma_commit(&s_full[j & 1]);
+        }
+        __syncwarp();
+      }
+    }
+    if (elect_one()) mma_commit(mma_done);
+    __syncwarp();
+    mbar_drain(mma_done, 0);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ P, dS, dQ epilogue
+    const int h = (warp - 4) >> 2;   // key columns [64h, 64h + 64) of every key tile
+    const int wq = warp & 3;         // 32-lane TMEM slice of this warp
+    const int row = wq * 32 + lane;  // query row within the tile
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const bool live = qt * kT + row < nq;  // padding rows of a ragged tile: zero terms, not stored
+    const size_t grow = grow0 + row;
+    // P = exp2(scale log2(e) q.k - log2(e) LSE); rows that see no key have
+    // every key masked (their -log2(e) LSE is stored as 0).
+    const float nl = live ? nlse2[grow] : 0.f;
+    const float dr = live ? dvec[grow] : 0.f;
+    const float2 c2 = make_float2(scale_log2, scale_log2), nl2 = make_float2(nl, nl);
+    bool ok = true;
+    for (int j = 0; ok && j < n; ++j) {
+      const int b = j & 1;
+      const uint32_t s_col = t_row + L::kColS + 128 * b + 64 * h;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // Keys past nk (ragged last tile) and, causal, keys after query + off
+      // get P = 0: key column c is kept iff c <= lim.
+      const int kv_valid = nk - j * kT;
+      const int diag_lim = (qt - j) * kT + off;
+      const bool masked = (CAUSAL && diag_lim < kT - 1) || kv_valid < kT;
+      int lim = kv_valid - 1;
+      if (CAUSAL && diag_lim + row < lim) lim = diag_lim + row;
+      float p[64];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld32(s_col + 32 * c, r);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 a = fma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nl2);
+          p[32 * c + 2 * i] = ex2(a.x);
+          p[32 * c + 2 * i + 1] = ex2(a.y);
+        }
+      }
+      if (masked) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (64 * h + i > lim) p[i] = 0.f;
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // dS = P (dP - D), 16-bit, into the S buffer's columns [64h, 64h + 32)
+      // (keys 2i, 2i + 1 of the warpgroup in column i), whose scores are in
+      // registers by now.
+      const float2 nd2 = make_float2(-dr, -dr);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_row + L::kColDP + 64 * h + 32 * c, r);
+        if (c == 1) {  // dP is in registers: dP(j+1) may overwrite it
+          tc_fence_before();
+          mbar_arrive(dp_read);
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 dpm = add2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), nd2);
+          const float2 ds = mul2(make_float2(p[32 * c + 2 * i], p[32 * c + 2 * i + 1]), dpm);
+          pk[i] = pack2<BF16>(ds.x, ds.y);
+        }
+        tmem_st16(s_col + 16 * c, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    // Epilogue: dQ = scale * (the accumulator); this warpgroup writes its
+    // half of the head dimension.
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dq_done, 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      uint4* dst = reinterpret_cast<uint4*>(dq_ptr + grow * D + (D / 2) * h);
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_row + L::kColDQ + (D / 2) * h + 32 * c, r);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * scale, __uint_as_float(r[2 * i + 1]) * scale);
+        if (live) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace attn

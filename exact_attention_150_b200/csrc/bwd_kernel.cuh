@@ -79,8 +79,8 @@ struct BwdLayout {
   static constexpr int kBExtBytes = kBwdTile * 16;
   static constexpr int kBarOff = kBExtOff + kBExtBytes;
   // kv_full, qd_full[S], qd_empty[S], s_full, dp_full, p_full, ds_full, dq_full, dq_free, acc_full, mma_done,
-  // bext_full, bext_free
-  static constexpr int kNumBars = 1 + 2 * kStages + 10;
+  // bext_full, bext_free, dp_read
+  static constexpr int kNumBars = 1 + 2 * kStages + 11;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   // The tiles need a 1024-byte aligned base.  The dynamic shared window
@@ -114,9 +114,11 @@ __global__ void __launch_bounds__(256)
       acc = fmaf(x.x, y.x, acc);
       acc = fmaf(x.y, y.y, acc);
     }
-    float4* z = reinterpret_cast<float4*>(dqacc + off);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (dqacc != nullptr) {  // the atomic-dQ backward accumulates into it
+      float4* z = reinterpret_cast<float4*>(dqacc + off);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
   for (int m = kTpr / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
@@ -191,40 +193,18 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Deterministic dQ: waits until *turn >= target (acquire), with the same
-// time limit and abort protocol as the mbarrier waits.
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ bool wait_turn(const int* turn, int target, volatile int* abort) {
-  if (ld_acquire_gpu(turn) >= target) return true;
-  const unsigned long long t0 = global_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i) {
-      __nanosleep(64);
-      if (ld_acquire_gpu(turn) >= target) return true;
-    }
-    if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      atomicExch(&g_device_status, kStatusTimeout);
-      return false;
-    }
-  }
-}
-
-template <int D, bool BF16, bool CAUSAL, bool DET>
+// DQ = true: the dQ contributions are formed here and added into the fp32
+// accumulator with atomics.  DQ = false: this kernel writes dK and dV only,
+// and bwd_dq_kernel computes dQ on its own (the reproducible backward).
+// max_qtiles: query tiles of the longest sequence (packed batches).
+template <int D, bool BF16, bool CAUSAL, bool DQ>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const float* __restrict__ dvec, const float* __restrict__ nlse2, float* __restrict__ dqacc,
-                    uint16_t* __restrict__ dk_ptr, uint16_t* __restrict__ dv_ptr, int* __restrict__ dq_order,
-                    const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H, int Nq, int Nk,
-                    int bottom_right, int order_stride, float scale, float scale_log2, int problems,
-                    int grid_tiles, int group) {
+                    uint16_t* __restrict__ dk_ptr, uint16_t* __restrict__ dv_ptr, const int* __restrict__ cu_q,
+                    const int* __restrict__ cu_k, int H, int Nq, int Nk, int bottom_right, int max_qtiles,
+                    float scale, float scale_log2, int problems, int grid_tiles, int group) {
   using L = BwdLayout<D>;
   constexpr bool kDqT = (D == 128);  // dQ formed transposed (see above)
   constexpr uint32_t kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 256 + D;
@@ -245,6 +225,7 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* mma_done = s_full + 7;
   uint64_t* bext_full = s_full + 8;  // warp 3 -> MMA: B_ext holds the current tile's terms
   uint64_t* bext_free = s_full + 9;  // MMA -> warp 3: the dP^T product has read B_ext
+  uint64_t* dp_read = s_full + 10;   // softmax -> MMA: dP^T loaded (DQ = false)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -269,9 +250,8 @@ __global__ void __launch_bounds__(512, 1)
     nk = clamp(cu_k[b + 1], Nk) - k0;
     nq = nq < 0 ? 0 : nq;
     nk = nk < 0 ? 0 : nk;
-    // Rows past max_seqlen_q (the grid's query tiles) are not computed; this
-    // also keeps the order counters of the deterministic mode in range.
-    nq = nq < order_stride * kBwdTile ? nq : order_stride * kBwdTile;
+    // Rows past max_seqlen_q (the grid's query tiles) are not computed.
+    nq = nq < max_qtiles * kBwdTile ? nq : max_qtiles * kBwdTile;
   }
   // Key tile j; causal: small j has the most work and launches first.
   if (j * kBwdTile >= nk) return;  // a sequence shorter than the grid
@@ -321,6 +301,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(mma_done, 1);
     mbar_init(bext_full, 32);
     mbar_init(bext_free, 1);
+    mbar_init(dp_read, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -419,33 +400,42 @@ __global__ void __launch_bounds__(512, 1)
       }
       mma_ss(tmem, ext_s, ext_b, kIdS, zero_scale ? 0u : 1u);
     };
+    auto issue_dp = [&](int it) {  // dP'^T of query tile it, then its commits
+      const uint64_t dod_k = sdesc_sw128(stage_addr(it) + L::kTileBytes, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        mma_ss(tmem + kColDP, kd_v + kmaj(ks), dod_k + kmaj(ks), kIdS, ks > 0 ? 1u : 0u);
+      mma_ss(tmem + kColDP, ext_d, ext_b, kIdS, 1u);
+      mma_commit(dp_full);
+      mma_commit(bext_free);  // S^T and dP^T of this tile have read B_ext
+    };
+    // Issue order per query tile it (DQ): dP^T(it) once the dQ drain has
+    // read the columns it reuses, dV(it), S^T(it+1), dK(it), dQ(it).
+    // Without dQ the dP^T columns hold nothing else, so dP^T(it+1) follows
+    // S^T(it+1) as soon as the dS pass has loaded dP^T(it):
+    //   dV(it), S^T(it+1), dP^T(it+1), dK(it).
     bool ok = wait_all(kv_full, 0) && wait_all(&qd_full[0], 0) && wait_all(bext_full, 0);
     if (ok && n_it > 0) {
       tc_fence_after();
       if (elect_one()) {
         issue_st(stage_addr(0));
         mma_commit(s_full);
+        if constexpr (!DQ) issue_dp(0);
       }
       __syncwarp();
     }
     for (int it = 0; ok && it < n_it; ++it) {
       const uint32_t q_addr = stage_addr(it);
       const uint32_t do_addr = q_addr + L::kTileBytes;
-      const uint64_t dod_k = sdesc_sw128(do_addr, 16, 1024);
       const uint64_t dod_mn = sdesc_sw128(do_addr, L::kChunkBytes, 1024);
       const uint64_t qd_mn = sdesc_sw128(q_addr, L::kChunkBytes, 1024);
-      // dP^T overwrites the previous tile's dQ columns: wait for the drain.
-      if (it > 0 && !(ok = wait_all(dq_free, (it - 1) & 1))) break;
-      tc_fence_after();
-      if (elect_one()) {
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          mma_ss(tmem + kColDP, kd_v + kmaj(ks), dod_k + kmaj(ks), kIdS, ks > 0 ? 1u : 0u);
-        mma_ss(tmem + kColDP, ext_d, ext_b, kIdS, 1u);
-        mma_commit(dp_full);
-        mma_commit(bext_free);  // S^T and dP^T of this tile have read B_ext
+      if constexpr (DQ) {
+        // dP^T overwrites the previous tile's dQ columns: wait for the drain.
+        if (it > 0 && !(ok = wait_all(dq_free, (it - 1) & 1))) break;
+        tc_fence_after();
+        if (elect_one()) issue_dp(it);
+        __syncwarp();
       }
-      __syncwarp();
       if (!(ok = wait_all(p_full, it & 1))) break;
       tc_fence_after();
       if (elect_one()) {
@@ -467,6 +457,12 @@ __global__ void __launch_bounds__(512, 1)
           mma_commit(s_full);
         }
         __syncwarp();
+        if constexpr (!DQ) {
+          if (!(ok = wait_all(dp_read, it & 1))) break;
+          tc_fence_after();
+          if (elect_one()) issue_dp(it + 1);
+          __syncwarp();
+        }
       }
       if (!(ok = wait_all(ds_full, it & 1))) break;
       tc_fence_after();
@@ -477,14 +473,16 @@ __global__ void __launch_bounds__(512, 1)
           mma_ss(tmem + kColDK, kd_ds + kmaj(ks), qd_mn + 128 * ks, kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&qd_empty[it % L::kStages]);
         if (it == n_it - 1) mma_commit(acc_full);
+        if constexpr (DQ) {
 #pragma unroll
-        for (int ks = 0; ks < kBwdTile / 16; ++ks) {
-          if constexpr (kDqT)  // A = K^T (M = d), B = dS^T (N = queries)
-            mma_ss(tmem + kColDQ, mn_k + 128 * ks, mn_ds + 128 * ks, kIdQ, ks > 0 ? 1u : 0u);
-          else  // A = dS (M = queries), B = K (N = d)
-            mma_ss(tmem + kColDQ, mn_ds + 128 * ks, mn_k + 128 * ks, kIdQ, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < kBwdTile / 16; ++ks) {
+            if constexpr (kDqT)  // A = K^T (M = d), B = dS^T (N = queries)
+              mma_ss(tmem + kColDQ, mn_k + 128 * ks, mn_ds + 128 * ks, kIdQ, ks > 0 ? 1u : 0u);
+            else  // A = dS (M = queries), B = K (N = d)
+              mma_ss(tmem + kColDQ, mn_ds + 128 * ks, mn_k + 128 * ks, kIdQ, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(dq_full);
         }
-        mma_commit(dq_full);
       }
       __syncwarp();
     }
@@ -596,6 +594,12 @@ __global__ void __launch_bounds__(512, 1)
       for (int c = 0; c < 2; ++c) {
         uint32_t pr[32];
         tmem_ld32(t_row + kColDP + 64 * h + 32 * c, pr);
+        if constexpr (!DQ) {
+          if (c == 1) {  // dP^T is in registers: the next tile's dP^T may overwrite it
+            tc_fence_before();
+            mbar_arrive(dp_read);
+          }
+        }
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           uint32_t dpk[8];
@@ -624,34 +628,11 @@ __global__ void __launch_bounds__(512, 1)
     const int row = wq * 32 + lane;  // TMEM lane: head-dim index (dQ^T) or query row (dQ)
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
+    for (int it = 0; DQ && it < n_it; ++it) {
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       const size_t qrow0 = qslab + static_cast<size_t>(i0 + it) * kBwdTile;
-      // Deterministic mode: the key tiles that reach a query tile are a
-      // prefix 0..J of the key tiles (the first query tile a key tile sees
-      // never decreases with it), so this CTA is contributor number j of
-      // every query tile it covers.  It reduces into the tile only after the
-      // 4 drain warps of contributors 0..j-1 have each counted theirs.
-      int* turn = DET ? dq_order + static_cast<size_t>(px) * order_stride + (i0 + it) : nullptr;
-      auto await_turn = [&]() {
-        if constexpr (DET) {
-          if (!__all_sync(0xffffffffu, wait_turn(turn, 4 * j, abort_flag))) return false;
-          __threadfence();
-        }
-        return true;
-      };
-      auto pass_turn = [&]() {
-        if constexpr (DET) {
-          __threadfence();
-          __syncwarp();
-          if (lane == 0) {
-            __threadfence();
-            atomicAdd(turn, 1);
-          }
-        }
-      };
       if constexpr (kDqT) {
         // Thread = head-dim index d; a warp's reduction covers 32 consecutive
         // d of one query row (128 contiguous bytes).
@@ -667,8 +648,6 @@ __global__ void __launch_bounds__(512, 1)
         tmem_ld32(t_row + kColDQ + 96, vd);
         tc_fence_before();
         mbar_arrive(dq_free);
-        ok = await_turn();
-        if (!ok) break;
 #pragma unroll
         for (int q = 0; q < 32; ++q)
           atomicAdd(base + static_cast<size_t>(q) * D, __uint_as_float(va[q]) * scale);
@@ -681,7 +660,6 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int q = 0; q < 32; ++q)
           atomicAdd(base + static_cast<size_t>(96 + q) * D, __uint_as_float(vd[q]) * scale);
-        pass_turn();
       } else {
         // Thread = query row; 64 head-dim values as 16-byte vector reductions.
         uint32_t va[32], vb[32];
@@ -689,8 +667,6 @@ __global__ void __launch_bounds__(512, 1)
         tmem_ld32(t_row + kColDQ + 32, vb);
         tc_fence_before();
         mbar_arrive(dq_free);
-        ok = await_turn();
-        if (!ok) break;
         float* dst = dqacc + (qrow0 + row) * D;
 #pragma unroll
         for (int v = 0; v < 8; ++v)
@@ -702,7 +678,6 @@ __global__ void __launch_bounds__(512, 1)
           atomicAdd(reinterpret_cast<float4*>(dst + 32 + 4 * v),
                     make_float4(__uint_as_float(vb[4 * v]) * scale, __uint_as_float(vb[4 * v + 1]) * scale,
                                 __uint_as_float(vb[4 * v + 2]) * scale, __uint_as_float(vb[4 * v + 3]) * scale));
-        pass_turn();
       }
     }
     if (ok && n_it > 0) {

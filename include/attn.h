@@ -151,8 +151,9 @@ attn_status attn_fwd_fp8_varlen(const void* q, const void* k, const void* v, voi
  * (128 - Nq % 128) % 128 rows of d floats of padding (a ragged last query
  * tile reduces its masked rows, which are exact zeros, into them), then the
  * fp32 row term D [B][H][Nq], then the fp32 row term -log2(e) * LSE
- * [B][H][Nq], then (16-byte aligned) B*H*ceil(Nq/128) int32 counters that
- * order the deterministic backward's dQ reductions.  Returns 0 for an empty
+ * [B][H][Nq], then (16-byte aligned) B*H*ceil(Nq/128) int32 words that no
+ * call uses at present (kept so that the size stays as documented).  Returns
+ * 0 for an empty
  * problem (any size 0), a negative size, or a total that overflows size_t.
  */
 size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d);
@@ -188,13 +189,16 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
  * attn_bwd with a bit-reproducible dQ.  The backward the pages describe has
  * no such variant; the page "Flash Attention 落地评估" (section 4) raises
  * reproducibility as a concern, and attn_bwd's dQ depends on the order in
- * which fp32 atomic additions from different key tiles land.  Here the key
- * tiles that reach a query tile add their dQ contributions in ascending
- * key-tile order (each waits, with the same bounded wait as every other wait
- * in these kernels, for a per-query-tile counter in the workspace), so two
- * calls with the same inputs give identical dQ, dK and dV bits.  It is slower
- * than attn_bwd: a key tile's reductions wait for the previous key tile's.
- * Arguments, workspace and errors as for attn_bwd.
+ * which fp32 atomic additions from different key tiles land.  Here dK and dV
+ * come from the same per-key-tile kernel as in attn_bwd (without its dQ
+ * product), and dQ from a second kernel with one CTA per query tile that
+ * recomputes the probabilities of each key tile it sees and accumulates its
+ * own dQ rows in order; nothing is added atomically, so two calls with the
+ * same inputs give identical dQ, dK and dV bits.  The second kernel repeats
+ * the S and dP products (7 matrix products per tile pair instead of 5), so
+ * it is somewhat slower than attn_bwd.  The dQ accumulator and the order
+ * counters of the workspace are not used.  Arguments, workspace and errors
+ * as for attn_bwd.
  */
 attn_status attn_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
                                    const float* lse, const void* dout, void* dq, void* dk, void* dv,
