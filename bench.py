@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload long_ctx] [--seq N] [--no-cpu-baseline] [--e2e-steps E]
-                    [--deterministic] [--varlen] [--fp8] [--e2e-pipelined [--e2e-chunks C]]
+                    [--deterministic] [--varlen] [--fp8] [--e2e-serial] [--e2e-chunks C]
 
 One step is one pass of the whole hot path over one batch of synthetic input:
 the forward kernel, then the three backward kernels (D preprocess, main,
@@ -24,11 +24,13 @@ attn_bwd_varlen on a seeded length mix; see workloads.VARLEN_MIX).
 per-tensor descales; see workloads.FWD_FP8), against an 8-bit peak of twice
 the measured bf16 peak (the nominal dense ratio).
 
-The e2e leg copies the step's inputs from pinned host memory, runs it and
-copies every result back, each step.  By default the copies and the calls
-run in order on one stream; --e2e-pipelined runs it through attn_host_step
-instead, which overlaps the copies of one chunk of (batch, head) slices with
-the kernels of another.
+The e2e leg runs the step end to end through the library's public call for
+host-resident tensors, attn_host_step: every step it copies the inputs from
+pinned host memory to the device, runs the forward and backward kernels and
+copies every result back, with the copies of one chunk of (batch, head)
+slices overlapping the kernels of another.  --e2e-serial instead copies the
+inputs, calls attn_fwd / attn_bwd and copies the results back in order on
+one stream.  Forward-only workloads always take the serial form.
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on a
 bounded sample of the same workload on the host cores, and prints the same
@@ -72,10 +74,10 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--varlen", action="store_true", help="time a packed variable-length batch")
     p.add_argument("--fp8", action="store_true", help="time the FP8 (E4M3) forward")
-    p.add_argument("--e2e-pipelined", action="store_true",
-                   help="run the e2e leg through attn_host_step (copies of one chunk of slices overlap the "
-                        "kernels of another); forward+backward workloads only")
-    p.add_argument("--e2e-chunks", type=int, default=4, help="chunks of (batch, head) slices for --e2e-pipelined")
+    p.add_argument("--e2e-serial", action="store_true",
+                   help="run the e2e leg as copies, attn_fwd, attn_bwd, copies in order on one stream instead of "
+                        "through attn_host_step")
+    p.add_argument("--e2e-chunks", type=int, default=4, help="chunks of (batch, head) slices of attn_host_step")
     p.add_argument("--deterministic", action="store_true",
                    help="time the bit-reproducible backward (attn_bwd_deterministic) instead of attn_bwd")
     return p.parse_args(argv)
@@ -168,6 +170,38 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
 def aggregate(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
     """Whole-job TFLOP/s: every rank processes `steps` steps of its replica."""
     return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
+def call_overhead(call, stream, n_host=200, n_graph=50, replays=10) -> dict:
+    """Where the time of a short call goes: the host's cost to validate,
+    encode the tensor maps and enqueue one call (wall clock over n_host calls,
+    the device idle or ahead), and the device time of one call with no host
+    gaps (a CUDA graph of n_graph calls, replayed)."""
+    import torch
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(n_host):
+        call()
+    t1 = time.perf_counter()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for _ in range(n_graph):
+                call()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(replays):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    return {"host_us_per_call": 1e6 * (t1 - t0) / n_host,
+            "graph_us_per_call": 1e3 * a.elapsed_time(b) / (replays * n_graph)}
 
 
 def sample_flops(w, rows) -> float:
@@ -446,6 +480,8 @@ def run_ours(args):
             kinfo["frac"] = kinfo["tflops"] / peak
     achieved = dom_flops / dom_ms / 1e9
     traffic = None if args.deterministic else KERNEL_TRAFFIC.get((w.name, w.N), {}).get(dom_name)
+    if fwd_ms < 0.1:
+        kernels["fwd_kernel"].update(call_overhead(fwd, stream))
 
     # End to end through the public API: pinned host inputs -> device, the
     # forward and backward calls, results -> pinned host, every step.
@@ -466,7 +502,8 @@ def run_ours(args):
             for dst, src in zip(outs_h, (o, lse, dq, dk, dv)):
                 dst.copy_(src, non_blocking=True)
 
-        if args.e2e_pipelined and w.backward:
+        pipelined = w.backward and not args.e2e_serial
+        if pipelined:
             # The same step through attn_host_step: the library copies every
             # chunk in, runs its kernels and copies its results out, with the
             # copies of one chunk overlapping the kernels of another.
@@ -494,7 +531,7 @@ def run_ours(args):
         e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, device)
         e2e = {"value": aggregate(step_flops, args.e2e_steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "path": (f"attn_host_step, {args.e2e_chunks} chunks" if args.e2e_pipelined and w.backward
+               "path": (f"attn_host_step, {args.e2e_chunks} chunks" if pipelined
                         else "copies, attn_fwd%s, copies on one stream" % (", attn_bwd" if w.backward else ""))}
 
     cpu = None
