@@ -58,8 +58,11 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of a kernel,
 # measured by ncu on this bench's command, keyed by (workload name, N) and
 # kernel.  Only valid for the kernel version it was taken on: remove an entry
-# when its kernel changes.
-KERNEL_TRAFFIC: dict = {}
+# when its kernel changes.  long_ctx: the full-set capture of the first timed
+# step of `bench.py --steps 2 --warmup 1 --e2e-steps 0 --no-cpu-baseline`.
+KERNEL_TRAFFIC: dict = {
+    ("long_ctx", 16384): {"bwd_main_kernel": 405_126_400 + 229_903_104, "fwd_kernel": 202_349_568 + 49_924_864},
+}
 
 
 def parse_args(argv=None):
@@ -77,7 +80,7 @@ def parse_args(argv=None):
     p.add_argument("--e2e-serial", action="store_true",
                    help="run the e2e leg as copies, attn_fwd, attn_bwd, copies in order on one stream instead of "
                         "through attn_host_step")
-    p.add_argument("--e2e-chunks", type=int, default=4, help="chunks of (batch, head) slices of attn_host_step")
+    p.add_argument("--e2e-chunks", type=int, default=8, help="chunks of (batch, head) slices of attn_host_step")
     p.add_argument("--deterministic", action="store_true",
                    help="time the bit-reproducible backward (attn_bwd_deterministic) instead of attn_bwd")
     return p.parse_args(argv)
