@@ -20,20 +20,23 @@
 //   warps 4-7    P and dS for key columns [0, 64) of every key tile
 //   warps 8-11   P and dS for key columns [64, 128)
 //                (thread = query row = TMEM lane: a row's LSE and D are
-//                per-thread values; each warpgroup also writes half of the
-//                head dimension of dQ at the end)
-// Tensor memory (512 columns):
-//   [0, 128), [128, 256)  S of even / odd key tiles (fp32); dS of the tile is
-//                         written in place, 16-bit packed, keys [64h, 64h+64)
-//                         in columns [64h, 64h+32)
-//   [256, 384)            dP = dO V^T (fp32)
-//   [384, 384+D)          dQ accumulator (fp32)
-// Products per key tile j: S(j) = Q K_j^T and dP(j) = dO V_j^T with both
-// operands in shared memory, dQ += dS(j) K_j with dS from tensor memory.
-// Issue order: S(0), dP(0), S(1), then per j: dP(j+1) once the softmax warps
-// have read dP(j), dQ(j) once they have written dS(j), S(j+2) into the
-// buffer that dQ(j) has just read.  The softmax warps therefore always find
-// the next S and dP ready when they finish a tile.
+//                per-thread values; at the start each warpgroup copies half
+//                of the head dimension of Q and dO into tensor memory, and at
+//                the end writes half of the head dimension of dQ)
+// Tensor memory (512 columns at d = 128):
+//   [0, 128)        S (fp32)
+//   [128, 256)      dP = dO V^T (fp32); dS of the tile is written over it,
+//                   16-bit packed, keys [64h, 64h+64) in columns
+//                   128 + [64h, 64h+32)
+//   [256, 256+D)    dQ accumulator (fp32)
+//   then Q and dO, 16-bit pairs (D/2 columns each): the A operands of S and dP
+// Products per key tile j: S(j) = Q K_j^T and dP(j) = dO V_j^T with A from
+// tensor memory (only K_j or V_j is read from shared memory), and
+// dQ += dS(j) K_j with dS from tensor memory.  Issue order: S(0), dP(0), then
+// per j: S(j+1) as soon as the softmax warps have loaded S(j) into
+// registers, dQ(j) once they have written dS(j), dP(j+1) behind dQ(j) (which
+// reads the dS it overwrites).  The warps find S(j+1) ready when they finish
+// tile j and wait for dP(j+1) only while dQ(j) and dP(j+1) run.
 #pragma once
 
 #include "sm100.cuh"
@@ -53,17 +56,19 @@ struct BwdDqLayout {
   static constexpr int kDOOff = kQOff + kTileBytes;
   static constexpr int kRingOff = kDOOff + kTileBytes;
   static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-  // qd_full, kv_full[kSlots], kv_empty[kSlots], s_full[2], dp_full, dp_read,
-  // ds_full, dq_done, mma_done
+  // qd_full, kv_full[kSlots], kv_empty[kSlots], s_full, s_read, dp_full,
+  // ds_full, dq_done, mma_done, qd_tmem
   static constexpr int kNumBars = 1 + 2 * kSlots + 7;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024 <= 232448 ? kBytes + 1024 : 232448;
   static_assert(kBytes <= 232448, "shared memory budget");
-  static constexpr uint32_t kColS = 0;     // S buffer b at kColS + 128 b
-  static constexpr uint32_t kColDP = 256;
-  static constexpr uint32_t kColDQ = 384;
-  static_assert(kColDQ + D <= 512, "tensor memory budget");
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColDP = 128;
+  static constexpr uint32_t kColDQ = 256;
+  static constexpr uint32_t kColQ = kColDQ + D;      // Q, 16-bit pairs
+  static constexpr uint32_t kColDO = kColQ + D / 2;  // dO, 16-bit pairs
+  static_assert(kColDO + D / 2 <= 512, "tensor memory budget");
 };
 
 // dvec and nlse2 hold D_i and -log2(e) LSE_i per query row of the tensor
@@ -85,12 +90,13 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* qd_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + L::kSlots;
-  uint64_t* s_full = kv_empty + L::kSlots;  // [2], by key-tile parity
-  uint64_t* dp_full = s_full + 2;
-  uint64_t* dp_read = dp_full + 1;          // 256 arrivals: dP loaded by the softmax warps
-  uint64_t* ds_full = dp_read + 1;          // 256 arrivals: dS written
+  uint64_t* s_full = kv_empty + L::kSlots;
+  uint64_t* s_read = s_full + 1;            // 256 arrivals: S loaded by the softmax warps
+  uint64_t* dp_full = s_read + 1;
+  uint64_t* ds_full = dp_full + 1;          // 256 arrivals: dS written
   uint64_t* dq_done = ds_full + 1;
   uint64_t* mma_done = dq_done + 1;
+  uint64_t* qd_tmem = mma_done + 1;         // 256 arrivals: Q and dO copied into tensor memory
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -148,13 +154,13 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_read, 256);
     mbar_init(dp_full, 1);
-    mbar_init(dp_read, 256);
     mbar_init(ds_full, 256);
     mbar_init(dq_done, 1);
     mbar_init(mma_done, 1);
+    mbar_init(qd_tmem, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -203,7 +209,7 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // K-major x K-major
+    constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // A (TMEM) x K-major
     constexpr uint32_t kIdQ = idesc_f16(BF16, 128, D, false, true);     // dS (TMEM) x K MN-major
     const uint32_t ring_base = smem_u32(smem + L::kRingOff);
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
@@ -211,84 +217,70 @@ __global__ void __launch_bounds__(384, 1)
     };
     auto slot_addr = [&](int item) { return ring_base + (item % L::kSlots) * L::kTileBytes; };
     auto wait_item = [&](int item) { return wait_all(&kv_full[item % L::kSlots], (item / L::kSlots) & 1); };
-    const uint64_t qd = sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
-    const uint64_t dod = sdesc_sw128(smem_u32(smem + L::kDOOff), 16, 1024);
-    // A K-major SW128 operand steps 32 bytes per K step of 16 inside a
-    // 128-byte row, and one 16 KB chunk per 64 columns.
+    // B K-major SW128: 32 bytes per K step of 16 inside a 128-byte row, one
+    // 16 KB chunk per 64 columns; A from tensor memory: 8 columns per step.
     auto kstep = [](int ks) { return static_cast<uint64_t>(((ks >> 2) * L::kChunkBytes + (ks & 3) * 32) >> 4); };
-    auto issue_s = [&](int j) {  // S(j) = Q K_j^T into buffer j & 1
+    auto issue_s = [&](int j) {  // S(j) = Q K_j^T
       const uint64_t kd = sdesc_sw128(slot_addr(2 * j), 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
-        mma_ss(tmem + L::kColS + 128 * (j & 1), qd + kstep(ks), kd + kstep(ks), kIdS, ks > 0 ? 1u : 0u);
+        mma_ts(tmem + L::kColS, tmem + L::kColQ + 8 * ks, kd + kstep(ks), kIdS, ks > 0 ? 1u : 0u);
     };
     auto issue_dp = [&](int j) {  // dP(j) = dO V_j^T
       const uint64_t vd = sdesc_sw128(slot_addr(2 * j + 1), 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
-        mma_ss(tmem + L::kColDP, dod + kstep(ks), vd + kstep(ks), kIdS, ks > 0 ? 1u : 0u);
+        mma_ts(tmem + L::kColDP, tmem + L::kColDO + 8 * ks, vd + kstep(ks), kIdS, ks > 0 ? 1u : 0u);
     };
-    // dQ += dS(j) K_j: A = dS from buffer j & 1 (key step ks of 16 keys:
-    // keys [64h, 64h + 64) sit in columns [64h, 64h + 32), 8 per step),
-    // B = K_j MN-major (16 key rows of 128 bytes per step).
+    // dQ += dS(j) K_j: A = dS over dP (key step ks of 16 keys: keys
+    // [64h, 64h + 64) sit in columns [64h, 64h + 32), 8 per step), B = K_j
+    // MN-major (16 key rows of 128 bytes per step).
     auto issue_dq = [&](int j) {
       const uint64_t kmn = sdesc_sw128(slot_addr(2 * j), L::kChunkBytes, 1024);
 #pragma unroll
       for (int ks = 0; ks < kT / 16; ++ks) {
-        const uint32_t ds_col = tmem + L::kColS + 128 * (j & 1) + 64 * (ks >> 2) + 8 * (ks & 3);
+        const uint32_t ds_col = tmem + L::kColDP + 64 * (ks >> 2) + 8 * (ks & 3);
         mma_ts(tmem + L::kColDQ, ds_col, kmn + 128 * ks, kIdQ, (j > 0 || ks > 0) ? 1u : 0u);
       }
     };
-    bool ok = wait_all(qd_full, 0) && wait_item(0) && wait_item(1);
+    bool ok = wait_all(qd_tmem, 0) && wait_item(0) && wait_item(1);
     if (ok) {
       tc_fence_after();
       if (elect_one()) {
         issue_s(0);
-        mma_commit(&s_full[0]);
+        mma_commit(s_full);
         issue_dp(0);
         mma_commit(dp_full);
         mma_commit(&kv_empty[1 % L::kSlots]);  // V_0 read
       }
       __syncwarp();
     }
-    if (ok && n > 1 && (ok = wait_item(2))) {
-      tc_fence_after();
-      if (elect_one()) {
-        issue_s(1);
-        mma_commit(&s_full[1]);
-      }
-      __syncwarp();
-    }
     for (int j = 0; ok && j < n; ++j) {
       if (j + 1 < n) {
-        // dP(j+1) overwrites dP(j): the softmax warps have loaded it.
-        if (!(ok = wait_all(dp_read, j & 1))) break;
-        if (!(ok = wait_item(2 * j + 3))) break;
+        // S(j+1) overwrites S(j): the softmax warps have loaded it.
+        if (!(ok = wait_all(s_read, j & 1))) break;
+        if (!(ok = wait_item(2 * j + 2))) break;
         tc_fence_after();
         if (elect_one()) {
-          issue_dp(j + 1);
-          mma_commit(dp_full);
-          mma_commit(&kv_empty[(2 * j + 3) % L::kSlots]);  // V_{j+1} read
+          issue_s(j + 1);
+          mma_commit(s_full);
         }
         __syncwarp();
       }
       if (!(ok = wait_all(ds_full, j & 1))) break;
+      if (j + 1 < n && !(ok = wait_item(2 * j + 3))) break;
       tc_fence_after();
       if (elect_one()) {
         issue_dq(j);
         mma_commit(&kv_empty[(2 * j) % L::kSlots]);  // K_j read by S(j) and dQ(j)
         if (j == n - 1) mma_commit(dq_done);
+        if (j + 1 < n) {
+          issue_dp(j + 1);  // over dS(j), which dQ(j) (issued above) reads first
+          mma_commit(dp_full);
+          mma_commit(&kv_empty[(2 * j + 3) % L::kSlots]);  // V_{j+1} read
+        }
       }
       __syncwarp();
-      if (j + 2 < n) {
-        if (!(ok = wait_item(2 * j + 4))) break;
-        tc_fence_after();
-        if (elect_one()) {
-          issue_s(j + 2);  // into the buffer whose dS dQ(j) (issued above) consumes first
-          mma_commit(&s_full[j & 1]);
-        }
-        __syncwarp();
-      }
     }
     if (elect_one()) mma_commit(mma_done);
     __syncwarp();
@@ -306,11 +298,35 @@ __global__ void __launch_bounds__(384, 1)
     const float nl = live ? nlse2[grow] : 0.f;
     const float dr = live ? dvec[grow] : 0.f;
     const float2 c2 = make_float2(scale_log2, scale_log2), nl2 = make_float2(nl, nl);
-    bool ok = true;
+    // Q and dO -> tensor memory: this thread copies its row's half of the
+    // head dimension (16-byte units of the 128-byte swizzled tiles) as
+    // 32-bit words of two 16-bit values, the lowest index in the low bits.
+    bool ok = __all_sync(0xffffffffu, mbar_wait(qd_full, 0, abort_flag));
+    if (ok) {
+      constexpr bool kTwoChunks = L::kRowBytes == 256;  // each warpgroup copies one whole chunk
+      constexpr int kUnits = L::kRowBytes / 32;          // 16-byte units in half a row
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint8_t* src = smem + (m == 0 ? L::kQOff : L::kDOOff) + (kTwoChunks ? h * L::kChunkBytes : 0) + row * 128;
+        uint32_t w[4 * kUnits];
+#pragma unroll
+        for (int u = 0; u < kUnits; ++u) {
+          const int unit = (kTwoChunks ? u : kUnits * h + u) ^ (row & 7);
+          const uint4 v4 = *reinterpret_cast<const uint4*>(src + unit * 16);
+          w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
+        }
+        const uint32_t col = (m == 0 ? L::kColQ : L::kColDO) + (D / 4) * h;
+        if constexpr (kTwoChunks)
+          tmem_st32(t_row + col, w);
+        else
+          tmem_st16(t_row + col, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+    }
+    mbar_arrive(qd_tmem);
     for (int j = 0; ok && j < n; ++j) {
-      const int b = j & 1;
-      const uint32_t s_col = t_row + L::kColS + 128 * b + 64 * h;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       // Keys past nk (ragged last tile) and, causal, keys after query + off
@@ -324,7 +340,11 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
-        tmem_ld32(s_col + 32 * c, r);
+        tmem_ld32(t_row + L::kColS + 64 * h + 32 * c, r);
+        if (c == 1) {  // S is in registers: S(j+1) may overwrite it
+          tc_fence_before();
+          mbar_arrive(s_read);
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float2 a = fma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nl2);
@@ -340,26 +360,22 @@ __global__ void __launch_bounds__(384, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      // dS = P (dP - D), 16-bit, into the S buffer's columns [64h, 64h + 32)
-      // (keys 2i, 2i + 1 of the warpgroup in column i), whose scores are in
-      // registers by now.
+      // dS = P (dP - D), 16-bit, over dP: keys 2i, 2i + 1 of the warpgroup in
+      // column 128 + 64h + i.  The 64 dP values are loaded first, since the
+      // packed dS lands in the first half of the warpgroup's dP columns.
       const float2 nd2 = make_float2(-dr, -dr);
+      uint32_t r[64];
+      tmem_ld64(t_row + L::kColDP + 64 * h, r);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_row + L::kColDP + 64 * h + 32 * c, r);
-        if (c == 1) {  // dP is in registers: dP(j+1) may overwrite it
-          tc_fence_before();
-          mbar_arrive(dp_read);
-        }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float2 dpm = add2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), nd2);
+          const float2 dpm = add2(make_float2(__uint_as_float(r[32 * c + 2 * i]), __uint_as_float(r[32 * c + 2 * i + 1])), nd2);
           const float2 ds = mul2(make_float2(p[32 * c + 2 * i], p[32 * c + 2 * i + 1]), dpm);
           pk[i] = pack2<BF16>(ds.x, ds.y);
         }
-        tmem_st16(s_col + 16 * c, pk);
+        tmem_st16(t_row + L::kColDP + 64 * h + 16 * c, pk);
       }
       tmem_st_wait();
       tc_fence_before();

@@ -79,8 +79,8 @@ struct BwdLayout {
   static constexpr int kBExtBytes = kBwdTile * 16;
   static constexpr int kBarOff = kBExtOff + kBExtBytes;
   // kv_full, qd_full[S], qd_empty[S], s_full, dp_full, p_full, ds_full, dq_full, dq_free, acc_full, mma_done,
-  // bext_full, bext_free, dp_read
-  static constexpr int kNumBars = 1 + 2 * kStages + 11;
+  // bext_full, bext_free
+  static constexpr int kNumBars = 1 + 2 * kStages + 10;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   // The tiles need a 1024-byte aligned base.  The dynamic shared window
@@ -225,7 +225,6 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* mma_done = s_full + 7;
   uint64_t* bext_full = s_full + 8;  // warp 3 -> MMA: B_ext holds the current tile's terms
   uint64_t* bext_free = s_full + 9;  // MMA -> warp 3: the dP^T product has read B_ext
-  uint64_t* dp_read = s_full + 10;   // softmax -> MMA: dP^T loaded (DQ = false)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -301,7 +300,6 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(mma_done, 1);
     mbar_init(bext_full, 32);
     mbar_init(bext_free, 1);
-    mbar_init(dp_read, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -411,9 +409,9 @@ __global__ void __launch_bounds__(512, 1)
     };
     // Issue order per query tile it (DQ): dP^T(it) once the dQ drain has
     // read the columns it reuses, dV(it), S^T(it+1), dK(it), dQ(it).
-    // Without dQ the dP^T columns hold nothing else, so dP^T(it+1) follows
-    // S^T(it+1) as soon as the dS pass has loaded dP^T(it):
-    //   dV(it), S^T(it+1), dP^T(it+1), dK(it).
+    // Without dQ, dS^T is only the A operand of dK, so the dS pass writes it
+    // over dP^T in tensor memory (no shared-memory copy) and dK reads it
+    // from there:  dV(it), S^T(it+1), dK(it), dP^T(it+1).
     bool ok = wait_all(kv_full, 0) && wait_all(&qd_full[0], 0) && wait_all(bext_full, 0);
     if (ok && n_it > 0) {
       tc_fence_after();
@@ -457,22 +455,24 @@ __global__ void __launch_bounds__(512, 1)
           mma_commit(s_full);
         }
         __syncwarp();
-        if constexpr (!DQ) {
-          if (!(ok = wait_all(dp_read, it & 1))) break;
-          tc_fence_after();
-          if (elect_one()) issue_dp(it + 1);
-          __syncwarp();
-        }
       }
       if (!(ok = wait_all(ds_full, it & 1))) break;
       tc_fence_after();
       if (elect_one()) {
-        // dK += dS^T Q: A = dS^T K-major in shared memory, B = Q MN-major.
+        // dK += dS^T Q: A = dS^T (DQ: K-major in shared memory; otherwise
+        // packed over dP^T in tensor memory), B = Q MN-major.
 #pragma unroll
-        for (int ks = 0; ks < kBwdTile / 16; ++ks)
-          mma_ss(tmem + kColDK, kd_ds + kmaj(ks), qd_mn + 128 * ks, kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < kBwdTile / 16; ++ks) {
+          if constexpr (DQ)
+            mma_ss(tmem + kColDK, kd_ds + kmaj(ks), qd_mn + 128 * ks, kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
+          else
+            mma_ts(tmem + kColDK, tmem + kColDP + p_col(ks), qd_mn + 128 * ks, kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
+        }
         mma_commit(&qd_empty[it % L::kStages]);
         if (it == n_it - 1) mma_commit(acc_full);
+        if constexpr (!DQ) {
+          if (it + 1 < n_it) issue_dp(it + 1);  // over dS^T(it), which dK (issued above) reads first
+        }
         if constexpr (DQ) {
 #pragma unroll
           for (int ks = 0; ks < kBwdTile / 16; ++ks) {
@@ -586,40 +586,45 @@ __global__ void __launch_bounds__(512, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
-      // dS pass: dS^T = P^T * dP'^T, packed 16-bit into the 128-byte-
-      // swizzled shared tile (row r, 64 queries per 16 KB chunk).
+      // dS pass: dS^T = P^T * dP'^T, packed 16-bit.  DQ: into the 128-byte-
+      // swizzled shared tile (row r, 64 queries per 16 KB chunk), the
+      // operand of both dK and dQ.  Otherwise over dP^T in tensor memory,
+      // in the column layout of P^T (queries 2i, 2i + 1 of chunk c in
+      // column 64h + 16c + i), each chunk landing in columns already read.
       if (!__all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag))) break;
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pr[32];
         tmem_ld32(t_row + kColDP + 64 * h + 32 * c, pr);
-        if constexpr (!DQ) {
-          if (c == 1) {  // dP^T is in registers: the next tile's dP^T may overwrite it
-            tc_fence_before();
-            mbar_arrive(dp_read);
-          }
-        }
+        uint32_t dsk[16];
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          uint32_t dpk[8];
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
             const int x = 16 * g + e;
             const float2 d = mul2(unpack2<BF16>(ppk[16 * c + x / 2]),
                                   make_float2(__uint_as_float(pr[x]), __uint_as_float(pr[x + 1])));
-            dpk[e / 2] = pack2<BF16>(d.x, d.y);
+            dsk[8 * g + e / 2] = pack2<BF16>(d.x, d.y);
           }
+          if constexpr (DQ) {
 #pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const int unit = (4 * c + 2 * g + v) ^ (r & 7);
-            *reinterpret_cast<uint4*>(ds_row + unit * 16) =
-                make_uint4(dpk[4 * v], dpk[4 * v + 1], dpk[4 * v + 2], dpk[4 * v + 3]);
+            for (int v = 0; v < 2; ++v) {
+              const int unit = (4 * c + 2 * g + v) ^ (r & 7);
+              *reinterpret_cast<uint4*>(ds_row + unit * 16) =
+                  make_uint4(dsk[8 * g + 4 * v], dsk[8 * g + 4 * v + 1], dsk[8 * g + 4 * v + 2], dsk[8 * g + 4 * v + 3]);
+            }
           }
         }
+        if constexpr (!DQ) tmem_st16(t_row + kColDP + 64 * h + 16 * c, dsk);
       }
-      tc_fence_before();
-      fence_proxy_async_smem();
+      if constexpr (DQ) {
+        tc_fence_before();
+        fence_proxy_async_smem();
+      } else {
+        tmem_st_wait();
+        tc_fence_before();
+      }
       mbar_arrive(ds_full);
     }
   } else if (warp >= 12) {
