@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -87,6 +88,18 @@ attn_status check_common(int B, int H, int Nq, int Nk, int d, int causal, attn_d
   if (bh * tiles(Nq) > 0x7fffffffLL || bh * tiles(Nk) > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if (bh * Nq > (1LL << 40) || bh * Nk > (1LL << 40)) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
+}
+
+// Multiprocessor count of the current device (0 if it cannot be read),
+// read once per device.
+int sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64 && (n = cached[dev].load(std::memory_order_relaxed)) > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device):
@@ -208,9 +221,17 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
   // Every CTA of a problem streams its K and V.
   const int group = attn::order_group(2.0 * L::kRowBytes * avg_rows(pb.rows_k, pb), pb.problems);
-  const unsigned grid = static_cast<unsigned>(pb.problems) * static_cast<unsigned>(pb.qtiles);
+  // Persistent: one CTA per SM (the shared memory and the 512 tensor-memory
+  // columns allow no second), each walking its share of the query tiles.
+  const unsigned units = static_cast<unsigned>(pb.problems) * static_cast<unsigned>(pb.qtiles);
+  const unsigned sms = static_cast<unsigned>(sm_count());
+  if (sms == 0) return ATTN_ERR_CUDA;
+  const unsigned grid = units < sms ? units : sms;
+  // Causal grids with at least two units per CTA deal heavy and light tiles
+  // out in pairs (tile_order.h).
+  const int fold = CAUSAL && units >= 2u * sms ? 1 : 0;
   kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, pb.cu_q, pb.cu_k, pb.H, pb.rows_q,
-                                     pb.rows_k, pb.bottom_right, scale_log2, pb.problems, pb.qtiles, group,
+                                     pb.rows_k, pb.bottom_right, scale_log2, pb.problems, pb.qtiles, group, fold,
                                      o_scale);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

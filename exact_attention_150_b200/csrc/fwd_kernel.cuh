@@ -15,9 +15,16 @@
 // of the SM's shared-memory bandwidth; with A in tensor memory it needs half,
 // which leaves room for the TMA writes of the K/V ring.
 //
+// The grid is persistent: one CTA per SM walks a share of the query tiles
+// (unit_at in tile_order.h), so one tile's epilogue overlaps the next tile's
+// Q load and first products, and the K/V ring, the S buffers and every
+// barrier run on across tiles (their phases count over all of the CTA's key
+// tiles).  Short grids lose no time to a CTA's set-up (barriers, tensor
+// memory, descriptor prefetch) per tile.
+//
 // CTA layout (384 threads, one CTA per SM):
-//   warp 0       TMA producer: Q once, then K_0, K_1, V_0, K_2, V_1, ...
-//                through a ring of shared-memory slots
+//   warp 0       TMA producer: per query tile Q, then K_0, K_1, V_0, K_2,
+//                V_1, ... through a ring of shared-memory slots
 //   warp 1       MMA issuer (one thread)
 //   warp 2       tensor-memory allocation / release
 //   warps 4-7    softmax for key columns [0, 64) of every key tile
@@ -99,7 +106,7 @@ __global__ void __launch_bounds__(384, 1)
                const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o_ptr,
                float* __restrict__ lse_ptr, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H,
                int Nq, int Nk, int bottom_right, float scale_log2, int problems, int grid_tiles, int group,
-               float o_scale) {
+               int fold, float o_scale) {
   static_assert(!F8 || BF16, "the 8-bit forward writes bf16");
   using L = FwdLayout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
@@ -124,52 +131,61 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  // The problem of this CTA: slab z of the tensor maps ([z][Nq or Nk][D])
-  // and rows [q0, q0 + nq) / [k0, k0 + nk) of it.  Dense batches have one
-  // slab per (batch, head) and use all of it.  Packed variable-length
-  // batches have one slab per head and take sequence b's rows from the
-  // offsets, clamped to the slab: bad offsets can give wrong values but
-  // never address outside the tensors.
-  // The grid is one-dimensional, in the grouped launch order of
-  // tile_order.h: px is the problem, ty the query tile in launch order.
-  int px, ty;
-  grouped_order(blockIdx.x, problems, grid_tiles, group, &px, &ty);
-  int z = px, q0 = 0, k0 = 0, nq = Nq, nk = Nk;
-  if (cu_q != nullptr) {
-    const int b = px / H;
-    z = px - b * H;
-    auto clamp = [](int v, int hi) { return v < 0 ? 0 : (v > hi ? hi : v); };
-    q0 = clamp(cu_q[b], Nq);
-    k0 = clamp(cu_k[b], Nk);
-    nq = clamp(cu_q[b + 1], Nq) - q0;
-    nk = clamp(cu_k[b + 1], Nk) - k0;
-    nq = nq < 0 ? 0 : nq;
-    nk = nk < 0 ? 0 : nk;
-  }
-  const int nqt = (nq + kTile - 1) / kTile;  // the last tiles may be ragged
-  const int nkt = (nk + kTile - 1) / kTile;
-  if (ty >= nqt) return;  // a sequence shorter than the grid
-  // Causal: the heaviest query tiles are launched first.
-  const int qt = CAUSAL ? (nqt - 1 - ty) : ty;
-  // Key tiles this query tile sees.  Causal: query i sees key k iff
-  // k <= i + off (off = 0 top-left, nk - nq bottom-right).
-  const int off = bottom_right ? nk - nq : 0;
-  int n = nkt;
-  if (CAUSAL) {
-    const int last_row = qt * kTile + kTile - 1 < nq - 1 ? qt * kTile + kTile - 1 : nq - 1;
-    const int last_key = last_row + off < nk - 1 ? last_row + off : nk - 1;
-    n = last_key < 0 ? 0 : last_key / kTile + 1;
-  }
-  if (n == 0) {
-    // No row of this tile sees a key (bottom-right with nq > nk, or a
-    // sequence without keys): the softmax is empty, O = 0 and LSE = log 0.
-    const int rows = nq - qt * kTile < kTile ? nq - qt * kTile : kTile;
-    const size_t grow0 = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile;
-    for (int e = threadIdx.x; e < rows * D / 8; e += blockDim.x)
-      reinterpret_cast<uint4*>(o_ptr + grow0 * D)[e] = make_uint4(0u, 0u, 0u, 0u);
-    for (int e = threadIdx.x; e < rows; e += blockDim.x) lse_ptr[grow0 + e] = -INFINITY;
-    return;
-  }
+  // Work units.  A unit is one 128-row query tile of one problem: slab z of
+  // the tensor maps ([z][Nq or Nk][D]) and rows [q0, q0 + nq) / [k0, k0 + nk)
+  // of it.  Dense batches have one slab per (batch, head) and use all of it;
+  // packed variable-length batches have one slab per head and take sequence
+  // b's rows from the offsets, clamped to the slab (bad offsets can give
+  // wrong values but never address outside the tensors).  The grid is
+  // persistent (at most one CTA per SM) and deals the units of the launch
+  // order of tile_order.h (grid_tiles query tiles of each of `problems`
+  // problems, causal grids heaviest first) out by unit_at: the units in
+  // flight at any time are neighbours in that order, and with `fold` (causal
+  // grids) a CTA takes a heavy tile and a light one together.  Every role
+  // walks the same units and takes the same decisions.
+  const UnitPlan plan = unit_plan(problems, grid_tiles, group, fold);
+  const int slots = unit_slots(plan, gridDim.x);
+  auto unit_index = [&](int s) { return unit_at(plan, gridDim.x, blockIdx.x, s); };
+  struct Unit {
+    int z, q0, k0, nq, nk, qt, n, off;
+    bool live;  // false: past the end of a shorter sequence, nothing to do
+  };
+  auto unit_of = [&](int u) {
+    Unit w;
+    int px, ty;
+    grouped_order(static_cast<unsigned>(u), problems, grid_tiles, group, &px, &ty);
+    w.z = px;
+    w.q0 = 0;
+    w.k0 = 0;
+    w.nq = Nq;
+    w.nk = Nk;
+    if (cu_q != nullptr) {
+      const int b = px / H;
+      w.z = px - b * H;
+      auto clamp = [](int v, int hi) { return v < 0 ? 0 : (v > hi ? hi : v); };
+      w.q0 = clamp(cu_q[b], Nq);
+      w.k0 = clamp(cu_k[b], Nk);
+      w.nq = clamp(cu_q[b + 1], Nq) - w.q0;
+      w.nk = clamp(cu_k[b + 1], Nk) - w.k0;
+      w.nq = w.nq < 0 ? 0 : w.nq;
+      w.nk = w.nk < 0 ? 0 : w.nk;
+    }
+    const int nqt = (w.nq + kTile - 1) / kTile;  // the last tiles may be ragged
+    const int nkt = (w.nk + kTile - 1) / kTile;
+    w.live = ty < nqt;
+    // Causal: the heaviest query tiles come first.
+    w.qt = CAUSAL ? (nqt - 1 - ty) : ty;
+    // Key tiles this query tile sees.  Causal: query i sees key k iff
+    // k <= i + off (off = 0 top-left, nk - nq bottom-right).
+    w.off = bottom_right ? w.nk - w.nq : 0;
+    w.n = nkt;
+    if (CAUSAL && w.live) {
+      const int last_row = w.qt * kTile + kTile - 1 < w.nq - 1 ? w.qt * kTile + kTile - 1 : w.nq - 1;
+      const int last_key = last_row + w.off < w.nk - 1 ? last_row + w.off : w.nk - 1;
+      w.n = last_key < 0 ? 0 : last_key / kTile + 1;
+    }
+    return w;
+  };
 
   // Refuse to run (and report) if alignment left too little shared memory.
   if (static_cast<uint32_t>(smem - smem_raw) + L::kBytes > dynamic_smem_bytes()) {
@@ -218,30 +234,42 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(q_full, L::kTileBytes);
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_3d(smem + L::kQOff + c * L::kChunkBytes, &tm_q, q_full, c * L::kChunkElems, q0 + qt * kTile, z);
-      // Ring order: K_0, K_1, then V_j, K_{j+2} for j = 0, 1, ...
-      int item = 0;
+      int item = 0;  // ring position over all units
+      int uu = 0;    // units with key tiles whose Q load was issued
       bool ok = true;
-      auto load = [&](const CUtensorMap* map, int tile) {
-        const int slot = item % L::kSlots;
-        if (!mbar_wait(&kv_empty[slot], ((item / L::kSlots) & 1) ^ 1, abort_flag)) return false;
-        mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
-        uint8_t* dst = smem + L::kRingOff + slot * L::kTileBytes;
+      for (int r = 0; ok && r < slots; ++r) {
+        const int u = unit_index(r);
+        if (u < 0) continue;
+        const Unit w = unit_of(u);
+        if (!w.live || w.n == 0) continue;
+        // The Q buffer is free once the previous unit's Q has been copied
+        // into tensor memory (d = 256: once its S products are done).
+        if (uu > 0 && !(ok = mbar_wait(L::kWide ? o_full : q_tmem, (uu - 1) & 1, abort_flag))) break;
+        mbar_arrive_expect_tx(q_full, L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * L::kChunkElems, k0 + tile * kTile, z);
-        ++item;
-        return true;
-      };
-      for (int j = 0; ok && j < 2 && j < n; ++j) ok = load(&tm_k, j);
-      for (int j = 0; ok && j < n; ++j) {
-        ok = load(&tm_v, j);
-        if (ok && j + 2 < n) ok = load(&tm_k, j + 2);
+          tma_load_3d(smem + L::kQOff + c * L::kChunkBytes, &tm_q, q_full, c * L::kChunkElems,
+                      w.q0 + w.qt * kTile, w.z);
+        ++uu;  // Q loads issued
+        // Ring order: K_0, K_1, then V_j, K_{j+2} for j = 0, 1, ...
+        auto load = [&](const CUtensorMap* map, int tile) {
+          const int slot = item % L::kSlots;
+          if (!mbar_wait(&kv_empty[slot], ((item / L::kSlots) & 1) ^ 1, abort_flag)) return false;
+          mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
+          uint8_t* dst = smem + L::kRingOff + slot * L::kTileBytes;
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_3d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * L::kChunkElems, w.k0 + tile * kTile, w.z);
+          ++item;
+          return true;
+        };
+        for (int j = 0; ok && j < 2 && j < w.n; ++j) ok = load(&tm_k, j);
+        for (int j = 0; ok && j < w.n; ++j) {
+          ok = load(&tm_v, j);
+          if (ok && j + 2 < w.n) ok = load(&tm_k, j + 2);
+        }
       }
       if (!ok) {
         // Let the copies already issued land before the CTA exits.
-        mbar_drain(q_full, 0);
+        if (uu > 0) mbar_drain(q_full, (uu - 1) & 1);
         const int first = item > L::kSlots ? item - L::kSlots : 0;
         for (int i = first; i < item; ++i) mbar_drain(&kv_full[i % L::kSlots], (i / L::kSlots) & 1);
       }
@@ -310,45 +338,61 @@ __global__ void __launch_bounds__(384, 1)
       }
     };
 
-    bool ok = wait_all(q_tmem, 0);
-    for (int j = 0; ok && j < 2 && j < n; ++j) {
-      uint32_t ka;
-      if (!(ok = wait_slot(ka))) break;
-      tc_fence_after();
-      if (elect_one()) {
-        issue_s(j, ka);
-        mma_commit(&s_full[j]);
-        mma_commit(&kv_empty[item % L::kSlots]);
-      }
-      __syncwarp();
-      ++item;
-    }
-    for (int j = 0; ok && j < n; ++j) {
-      const int b = j & 1;
-      uint32_t va;
-      if (!(ok = wait_slot(va))) break;
-      if (!(ok = wait_all(&p_full[b], (j >> 1) & 1))) break;
-      tc_fence_after();
-      if (elect_one()) {
-        issue_pv(b, va, j > 0);
-        mma_commit(pv_done);
-        mma_commit(&kv_empty[item % L::kSlots]);
-        if (j == n - 1) mma_commit(o_full);
-      }
-      __syncwarp();
-      ++item;
-      if (j + 2 < n) {
+    // Key tiles run through the two S buffers in turn over all units: the
+    // g-th key tile of this CTA uses buffer g & 1.
+    int uu = 0, g = 0;  // units with key tiles, key tiles before the current unit
+    bool ok = true;
+    for (int r = 0; ok && r < slots; ++r) {
+      const int u = unit_index(r);
+      if (u < 0) continue;
+      const Unit w = unit_of(u);
+      if (!w.live || w.n == 0) continue;
+      const int n = w.n;
+      // Q of this unit is in tensor memory (d = 256: in shared memory).
+      if (!(ok = wait_all(q_tmem, uu & 1))) break;
+      for (int j = 0; ok && j < 2 && j < n; ++j) {
         uint32_t ka;
         if (!(ok = wait_slot(ka))) break;
         tc_fence_after();
         if (elect_one()) {
-          issue_s(b, ka);  // P(j) in this buffer was consumed by PV(j) above
-          mma_commit(&s_full[b]);
+          issue_s((g + j) & 1, ka);
+          mma_commit(&s_full[(g + j) & 1]);
           mma_commit(&kv_empty[item % L::kSlots]);
         }
         __syncwarp();
         ++item;
       }
+      for (int j = 0; ok && j < n; ++j) {
+        const int b = (g + j) & 1;
+        uint32_t va;
+        if (!(ok = wait_slot(va))) break;
+        if (!(ok = wait_all(&p_full[b], ((g + j) >> 1) & 1))) break;
+        tc_fence_after();
+        if (elect_one()) {
+          // j = 0 starts the unit's O and L afresh; the previous unit's
+          // epilogue has read them (its p_full follows that epilogue).
+          issue_pv(b, va, j > 0);
+          mma_commit(pv_done);
+          mma_commit(&kv_empty[item % L::kSlots]);
+          if (j == n - 1) mma_commit(o_full);
+        }
+        __syncwarp();
+        ++item;
+        if (j + 2 < n) {
+          uint32_t ka;
+          if (!(ok = wait_slot(ka))) break;
+          tc_fence_after();
+          if (elect_one()) {
+            issue_s(b, ka);  // P(j) in this buffer was consumed by PV(j) above
+            mma_commit(&s_full[b]);
+            mma_commit(&kv_empty[item % L::kSlots]);
+          }
+          __syncwarp();
+          ++item;
+        }
+      }
+      g += n;
+      ++uu;
     }
     if (elect_one()) mma_commit(mma_done);
     __syncwarp();
@@ -360,213 +404,238 @@ __global__ void __launch_bounds__(384, 1)
     const int row = wq * 32 + lane;  // query row within the tile
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
 
-    // Q -> TMEM: this thread copies its row's half of the head dimension
-    // (16-byte units of the 128-byte swizzled tile) as 32-bit words of two
-    // 16-bit or four 8-bit values, the lowest K index in the lowest bits.
-    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag));
-    if constexpr (!L::kWide) {  // d = 256: Q stays in shared memory
-      if (ok) {
-        constexpr bool kTwoChunks = L::kRowBytes == 256;  // each warpgroup copies one whole chunk
-        constexpr int kUnits = L::kRowBytes / 32;          // 16-byte units in half a row
-        const uint8_t* qrow = smem + L::kQOff + (kTwoChunks ? h * L::kChunkBytes : 0) + row * 128;
-        uint32_t qv[4 * kUnits];
+    const bool pos_scale = scale_log2 > 0.f;
+    const float cx = pos_scale ? scale_log2 : 1.f;
+    int uu = 0, g = 0;  // units with key tiles, key tiles before the current unit
+    bool ok = true;
+    for (int r = 0; ok && r < slots; ++r) {
+      const int u = unit_index(r);
+      if (u < 0) continue;
+      const Unit w = unit_of(u);
+      if (!w.live) continue;
+      const int z = w.z, q0 = w.q0, nq = w.nq, nk = w.nk, qt = w.qt, n = w.n, off = w.off;
+      if (n == 0) {
+        // No row of this tile sees a key (bottom-right with nq > nk, or a
+        // sequence without keys): the softmax is empty, O = 0 and LSE = log 0.
+        const int rows = nq - qt * kTile < kTile ? nq - qt * kTile : kTile;
+        const size_t grow0 = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile;
+        const int t0 = static_cast<int>(threadIdx.x) - 128;  // the 256 softmax threads
+        for (int e = t0; e < rows * D / 8; e += 256)
+          reinterpret_cast<uint4*>(o_ptr + grow0 * D)[e] = make_uint4(0u, 0u, 0u, 0u);
+        for (int e = t0; e < rows; e += 256) lse_ptr[grow0 + e] = -INFINITY;
+        continue;
+      }
+      // Q -> TMEM: this thread copies its row's half of the head dimension
+      // (16-byte units of the 128-byte swizzled tile) as 32-bit words of two
+      // 16-bit or four 8-bit values, the lowest K index in the lowest bits.
+      ok = __all_sync(0xffffffffu, mbar_wait(q_full, uu & 1, abort_flag));
+      if constexpr (!L::kWide) {  // d = 256: Q stays in shared memory
+        if (ok) {
+          constexpr bool kTwoChunks = L::kRowBytes == 256;  // each warpgroup copies one whole chunk
+          constexpr int kUnits = L::kRowBytes / 32;          // 16-byte units in half a row
+          const uint8_t* qrow = smem + L::kQOff + (kTwoChunks ? h * L::kChunkBytes : 0) + row * 128;
+          uint32_t qv[4 * kUnits];
 #pragma unroll
-        for (int u = 0; u < kUnits; ++u) {
-          const int unit = (kTwoChunks ? u : kUnits * h + u) ^ (row & 7);
-          const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + unit * 16);
-          qv[4 * u] = v4.x; qv[4 * u + 1] = v4.y; qv[4 * u + 2] = v4.z; qv[4 * u + 3] = v4.w;
+          for (int e = 0; e < kUnits; ++e) {
+            const int unit = (kTwoChunks ? e : kUnits * h + e) ^ (row & 7);
+            const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + unit * 16);
+            qv[4 * e] = v4.x; qv[4 * e + 1] = v4.y; qv[4 * e + 2] = v4.z; qv[4 * e + 3] = v4.w;
+          }
+          if constexpr (kTwoChunks) {
+            tmem_st32(t_row + L::kColQ + 32 * h, qv);
+          } else {
+            tmem_st16(t_row + L::kColQ + 16 * h, qv);
+          }
+          tmem_st_wait();
+          tc_fence_before();
         }
-        if constexpr (kTwoChunks) {
-          tmem_st32(t_row + L::kColQ + 32 * h, qv);
-        } else {
-          tmem_st16(t_row + L::kColQ + 16 * h, qv);
+      }
+
+      mbar_arrive(q_tmem);
+
+      float m_run = -INFINITY;  // running row max (log2 units; stale by < 8)
+      float l_run = 0.f;        // this warpgroup's part of sum exp2(score - m_run)
+      float lr_run = 0.f;       // d = 256: the same sum of the 16-bit rounded values
+
+      for (int j = 0; ok && j < n; ++j) {
+        const int gj = g + j;  // key tile count over all units of this CTA
+        const int b = gj & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (gj >> 1) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t s_col = t_row + L::kColS + 128 * b + 64 * h;
+        float x[64];
+        {
+          uint32_t r[64];
+          tmem_ld64(s_col, r);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(r[i]);
+        }
+        if (!pos_scale) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) x[c] *= scale_log2;
+        }
+        // Mask keys past nk (ragged last tile) and, causal, keys after
+        // query + off: column c is kept iff c <= lim.
+        const int kv_valid = nk - j * kTile;
+        const int diag_lim = (qt - j) * kTile + off;  // lim of row 0 from the mask
+        if ((CAUSAL && diag_lim < kTile - 1) || kv_valid < kTile) {
+          int lim = kv_valid - 1;
+          if (CAUSAL && diag_lim + row < lim) lim = diag_lim + row;
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (64 * h + c > lim) x[c] = -INFINITY;
+        }
+        float mp[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mp[i] = x[i];
+#pragma unroll
+        for (int c = 8; c < 64; c += 2) mp[(c >> 1) & 7] = max3f(mp[(c >> 1) & 7], x[c], x[c + 1]);
+        float mx = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+        // Exponentials, sums and the in-place 16-bit P of this warpgroup's 64
+        // columns against the maximum m_run.  l_run sums the fp32
+        // probabilities (for LSE); the tensor core sums the rounded 16-bit ones
+        // (L).  Arguments and sums as packed fp32x2; one pair in four goes to
+        // the FMA-pipe exponential, since MUFU throughput bounds them otherwise.
+        // A row that has seen no key yet (m_run = -inf; causal with off < 0)
+        // uses 0: its scores are all -inf, so p = 0 rather than NaN.
+        // (d = 256: the rounded ones are summed here too, in sr.  F8: P is
+        // rounded to E4M3, four keys per 32-bit column, so the 64 keys take
+        // 16 columns; the lazy rescale keeps P <= 2^8, inside E4M3's 448.)
+        float2 su[4], sr[4];
+  #define ATTN_EXP_STORE()                                                                            \
+    {                                                                                                 \
+      _Pragma("unroll") for (int i = 0; i < 4; ++i) su[i] = sr[i] = make_float2(0.f, 0.f);            \
+      const float m_use = m_run == -INFINITY ? 0.f : m_run;                                           \
+      const float2 cx2 = make_float2(cx, cx), negm2 = make_float2(-m_use, -m_use);                    \
+      if constexpr (F8) {                                                                             \
+        uint32_t pk[16];                                                                              \
+        _Pragma("unroll") for (int i = 0; i < 16; ++i) {                                              \
+          const float2 a0 = fma2(make_float2(x[4 * i], x[4 * i + 1]), cx2, negm2);                    \
+          const float2 a1 = fma2(make_float2(x[4 * i + 2], x[4 * i + 3]), cx2, negm2);                \
+          const float2 p0 = make_float2(ex2(a0.x), ex2(a0.y));                                        \
+          const float2 p1 = (i & 1) ? exp2_poly2(a1) : make_float2(ex2(a1.x), ex2(a1.y));             \
+          pk[i] = pack4_e4m3(p0.x, p0.y, p1.x, p1.y);                                                 \
+          su[(2 * i) & 3] = add2(su[(2 * i) & 3], p0);                                                \
+          su[(2 * i + 1) & 3] = add2(su[(2 * i + 1) & 3], p1);                                        \
+        }                                                                                             \
+        tmem_st16(s_col, pk);                                                                         \
+      } else {                                                                                        \
+      _Pragma("unroll") for (int c = 0; c < 2; ++c) {                                                 \
+        uint32_t pk[16];                                                                              \
+        _Pragma("unroll") for (int i = 0; i < 16; ++i) {                                              \
+          const float2 a = fma2(make_float2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), cx2, negm2);   \
+          const float2 p = ((i & 3) == 3) ? exp2_poly2(a) : make_float2(ex2(a.x), ex2(a.y));          \
+          pk[i] = pack2<BF16>(p.x, p.y);                                                              \
+          su[i & 3] = add2(su[i & 3], p);                                                             \
+          if constexpr (L::kWide) sr[i & 3] = add2(sr[i & 3], unpack2<BF16>(pk[i]));                  \
+        }                                                                                             \
+        tmem_st16(s_col + 16 * c, pk);                                                                \
+      }                                                                                               \
+      }                                                                                               \
+    }
+        // Row maximum over both halves of the key tile, exchanged through
+        // shared memory (double-buffered by tile parity: a warpgroup cannot
+        // rewrite a slot before the other has passed the next exchange, which
+        // it reaches only after reading the slot).
+        xchg[(b * 2 + h) * kTile + row] = mx;
+        mbar_arrive(&xmax_bar[b]);
+        // After the first tile, compute P against the current maximum while
+        // the other warpgroup's half arrives: it stands unless the maximum has
+        // grown by more than 2^8 (then it is recomputed below; P is not read
+        // before p_full).
+        if (j > 0) ATTN_EXP_STORE()
+        ok = __all_sync(0xffffffffu, mbar_wait(&xmax_bar[b], (gj >> 1) & 1, abort_flag));
+        if (!ok) break;
+        mx = fmaxf(mx, xchg[(b * 2 + (h ^ 1)) * kTile + row]);
+        const float m_new = fmaxf(m_run, mx * cx);
+        // Rescale O and the sums only when the maximum has grown by more than
+        // 2^8; otherwise keep the stale maximum (P stays below 256).  Both
+        // warpgroups see the same m_run and m_new, so they decide alike.
+        const bool need = (j > 0) && (m_new - m_run > 8.f);
+        if (j == 0) m_run = m_new;
+        const bool any_need = __any_sync(0xffffffffu, need);
+        if (any_need) {
+          // O must hold PV(j-1) complete before it is rescaled.
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (gj - 1) & 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+          const float alpha = need ? ex2(m_run - m_new) : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t r[32];
+            tmem_ld32(t_row + L::kColO + (D / 2) * h + 32 * c, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(t_row + L::kColO + (D / 2) * h + 32 * c, r);
+          }
+          if constexpr (!L::kWide) {
+            if (h == 0) tmem_st1(t_row + L::kColL, __float_as_uint(__uint_as_float(tmem_ld1(t_row + L::kColL)) * alpha));
+          }
+          if (need) {
+            l_run *= alpha;
+            lr_run *= alpha;
+            m_run = m_new;
+          }
+        }
+        // First tile, or a maximum that moved: (re)compute against the final
+        // m_run (rows of the warp whose m_run did not move get the same values).
+        if (j == 0 || any_need) {
+          if (j > 0) tmem_st_wait();  // the optimistic stores land before they are overwritten
+          ATTN_EXP_STORE()
+        }
+  #undef ATTN_EXP_STORE
+        const float2 su01 = add2(su[0], su[1]), su23 = add2(su[2], su[3]);
+        l_run += (su01.x + su01.y) + (su23.x + su23.y);
+        if constexpr (L::kWide) {
+          const float2 sr01 = add2(sr[0], sr[1]), sr23 = add2(sr[2], sr[3]);
+          lr_run += (sr01.x + sr01.y) + (sr23.x + sr23.y);
         }
         tmem_st_wait();
         tc_fence_before();
+        mbar_arrive(&p_full[b]);
       }
-    }
-    mbar_arrive(q_tmem);
-
-    const bool pos_scale = scale_log2 > 0.f;
-    const float cx = pos_scale ? scale_log2 : 1.f;
-    float m_run = -INFINITY;  // running row max (log2 units; stale by < 8)
-    float l_run = 0.f;        // this warpgroup's part of sum exp2(score - m_run)
-    float lr_run = 0.f;       // d = 256: the same sum of the 16-bit rounded values
-    for (int j = 0; ok && j < n; ++j) {
-      const int b = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t s_col = t_row + L::kColS + 128 * b + 64 * h;
-      float x[64];
-      {
-        uint32_t r[64];
-        tmem_ld64(s_col, r);
-#pragma unroll
-        for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(r[i]);
-      }
-      if (!pos_scale) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) x[c] *= scale_log2;
-      }
-      // Mask keys past nk (ragged last tile) and, causal, keys after
-      // query + off: column c is kept iff c <= lim.
-      const int kv_valid = nk - j * kTile;
-      const int diag_lim = (qt - j) * kTile + off;  // lim of row 0 from the mask
-      if ((CAUSAL && diag_lim < kTile - 1) || kv_valid < kTile) {
-        int lim = kv_valid - 1;
-        if (CAUSAL && diag_lim + row < lim) lim = diag_lim + row;
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (64 * h + c > lim) x[c] = -INFINITY;
-      }
-      float mp[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mp[i] = x[i];
-#pragma unroll
-      for (int c = 8; c < 64; c += 2) mp[(c >> 1) & 7] = max3f(mp[(c >> 1) & 7], x[c], x[c + 1]);
-      float mx = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
-      // Exponentials, sums and the in-place 16-bit P of this warpgroup's 64
-      // columns against the maximum m_run.  l_run sums the fp32
-      // probabilities (for LSE); the tensor core sums the rounded 16-bit ones
-      // (L).  Arguments and sums as packed fp32x2; one pair in four goes to
-      // the FMA-pipe exponential, since MUFU throughput bounds them otherwise.
-      // A row that has seen no key yet (m_run = -inf; causal with off < 0)
-      // uses 0: its scores are all -inf, so p = 0 rather than NaN.
-      // (d = 256: the rounded ones are summed here too, in sr.  F8: P is
-      // rounded to E4M3, four keys per 32-bit column, so the 64 keys take
-      // 16 columns; the lazy rescale keeps P <= 2^8, inside E4M3's 448.)
-      float2 su[4], sr[4];
-#define ATTN_EXP_STORE()                                                                            \
-  {                                                                                                 \
-    _Pragma("unroll") for (int i = 0; i < 4; ++i) su[i] = sr[i] = make_float2(0.f, 0.f);            \
-    const float m_use = m_run == -INFINITY ? 0.f : m_run;                                           \
-    const float2 cx2 = make_float2(cx, cx), negm2 = make_float2(-m_use, -m_use);                    \
-    if constexpr (F8) {                                                                             \
-      uint32_t pk[16];                                                                              \
-      _Pragma("unroll") for (int i = 0; i < 16; ++i) {                                              \
-        const float2 a0 = fma2(make_float2(x[4 * i], x[4 * i + 1]), cx2, negm2);                    \
-        const float2 a1 = fma2(make_float2(x[4 * i + 2], x[4 * i + 3]), cx2, negm2);                \
-        const float2 p0 = make_float2(ex2(a0.x), ex2(a0.y));                                        \
-        const float2 p1 = (i & 1) ? exp2_poly2(a1) : make_float2(ex2(a1.x), ex2(a1.y));             \
-        pk[i] = pack4_e4m3(p0.x, p0.y, p1.x, p1.y);                                                 \
-        su[(2 * i) & 3] = add2(su[(2 * i) & 3], p0);                                                \
-        su[(2 * i + 1) & 3] = add2(su[(2 * i + 1) & 3], p1);                                        \
-      }                                                                                             \
-      tmem_st16(s_col, pk);                                                                         \
-    } else {                                                                                        \
-    _Pragma("unroll") for (int c = 0; c < 2; ++c) {                                                 \
-      uint32_t pk[16];                                                                              \
-      _Pragma("unroll") for (int i = 0; i < 16; ++i) {                                              \
-        const float2 a = fma2(make_float2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), cx2, negm2);   \
-        const float2 p = ((i & 3) == 3) ? exp2_poly2(a) : make_float2(ex2(a.x), ex2(a.y));          \
-        pk[i] = pack2<BF16>(p.x, p.y);                                                              \
-        su[i & 3] = add2(su[i & 3], p);                                                             \
-        if constexpr (L::kWide) sr[i & 3] = add2(sr[i & 3], unpack2<BF16>(pk[i]));                  \
-      }                                                                                             \
-      tmem_st16(s_col + 16 * c, pk);                                                                \
-    }                                                                                               \
-    }                                                                                               \
-  }
-      // Row maximum over both halves of the key tile, exchanged through
-      // shared memory (double-buffered by tile parity: a warpgroup cannot
-      // rewrite a slot before the other has passed the next exchange, which
-      // it reaches only after reading the slot).
-      xchg[(b * 2 + h) * kTile + row] = mx;
-      mbar_arrive(&xmax_bar[b]);
-      // After the first tile, compute P against the current maximum while
-      // the other warpgroup's half arrives: it stands unless the maximum has
-      // grown by more than 2^8 (then it is recomputed below; P is not read
-      // before p_full).
-      if (j > 0) ATTN_EXP_STORE()
-      ok = __all_sync(0xffffffffu, mbar_wait(&xmax_bar[b], (j >> 1) & 1, abort_flag));
-      if (!ok) break;
-      mx = fmaxf(mx, xchg[(b * 2 + (h ^ 1)) * kTile + row]);
-      const float m_new = fmaxf(m_run, mx * cx);
-      // Rescale O and the sums only when the maximum has grown by more than
-      // 2^8; otherwise keep the stale maximum (P stays below 256).  Both
-      // warpgroups see the same m_run and m_new, so they decide alike.
-      const bool need = (j > 0) && (m_new - m_run > 8.f);
-      if (j == 0) m_run = m_new;
-      const bool any_need = __any_sync(0xffffffffu, need);
-      if (any_need) {
-        // O must hold PV(j-1) complete before it is rescaled.
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, abort_flag));
-        if (!ok) break;
+      // Epilogue: combine the two warpgroups' row sums, then each warpgroup
+      // writes its half of the head dimension of O.
+      xsum[h * kTile + row] = l_run;
+      if constexpr (L::kWide) xsum[(2 + h) * kTile + row] = lr_run;
+      mbar_arrive(xsum_bar);
+      if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(xsum_bar, uu & 1, abort_flag));
+      if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_full, uu & 1, abort_flag));
+      if (ok && n > 0) {
         tc_fence_after();
-        const float alpha = need ? ex2(m_run - m_new) : 1.f;
+        const float l_tot = l_run + xsum[(h ^ 1) * kTile + row];
+        // A row that sees no key keeps m_run = -inf: O = 0 and LSE = -inf.
+        // (Its sums are not exactly 0: the FMA-pipe exponential returns
+        // ~2^-126 rather than 0 for a masked score.)
+        // (tcgen05.ld is warp-collective: every lane loads, then selects.)
+        const bool empty = m_run == -INFINITY;
+        float l_tc;
+        if constexpr (L::kWide)
+          l_tc = lr_run + xsum[(2 + (h ^ 1)) * kTile + row];
+        else
+          l_tc = __uint_as_float(tmem_ld1(t_row + L::kColL));
+        const float inv = empty ? 0.f : (F8 ? o_scale : 1.f) / l_tc;
+        const bool live = qt * kTile + row < nq;  // padding rows of a ragged tile are not stored
+        const size_t grow = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile + row;
+        uint4* dst = reinterpret_cast<uint4*>(o_ptr + grow * D + (D / 2) * h);
 #pragma unroll 1
         for (int c = 0; c < D / 64; ++c) {
           uint32_t r[32];
           tmem_ld32(t_row + L::kColO + (D / 2) * h + 32 * c, r);
+          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(t_row + L::kColO + (D / 2) * h + 32 * c, r);
-        }
-        if constexpr (!L::kWide) {
-          if (h == 0) tmem_st1(t_row + L::kColL, __float_as_uint(__uint_as_float(tmem_ld1(t_row + L::kColL)) * alpha));
-        }
-        if (need) {
-          l_run *= alpha;
-          lr_run *= alpha;
-          m_run = m_new;
-        }
-      }
-      // First tile, or a maximum that moved: (re)compute against the final
-      // m_run (rows of the warp whose m_run did not move get the same values).
-      if (j == 0 || any_need) {
-        if (j > 0) tmem_st_wait();  // the optimistic stores land before they are overwritten
-        ATTN_EXP_STORE()
-      }
-#undef ATTN_EXP_STORE
-      const float2 su01 = add2(su[0], su[1]), su23 = add2(su[2], su[3]);
-      l_run += (su01.x + su01.y) + (su23.x + su23.y);
-      if constexpr (L::kWide) {
-        const float2 sr01 = add2(sr[0], sr[1]), sr23 = add2(sr[2], sr[3]);
-        lr_run += (sr01.x + sr01.y) + (sr23.x + sr23.y);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[b]);
-    }
-    // Epilogue: combine the two warpgroups' row sums, then each warpgroup
-    // writes its half of the head dimension of O.
-    xsum[h * kTile + row] = l_run;
-    if constexpr (L::kWide) xsum[(2 + h) * kTile + row] = lr_run;
-    mbar_arrive(xsum_bar);
-    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(xsum_bar, 0, abort_flag));
-    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort_flag));
-    if (ok && n > 0) {
-      tc_fence_after();
-      const float l_tot = l_run + xsum[(h ^ 1) * kTile + row];
-      // A row that sees no key keeps m_run = -inf: O = 0 and LSE = -inf.
-      // (Its sums are not exactly 0: the FMA-pipe exponential returns
-      // ~2^-126 rather than 0 for a masked score.)
-      // (tcgen05.ld is warp-collective: every lane loads, then selects.)
-      const bool empty = m_run == -INFINITY;
-      float l_tc;
-      if constexpr (L::kWide)
-        l_tc = lr_run + xsum[(2 + (h ^ 1)) * kTile + row];
-      else
-        l_tc = __uint_as_float(tmem_ld1(t_row + L::kColL));
-      const float inv = empty ? 0.f : (F8 ? o_scale : 1.f) / l_tc;
-      const bool live = qt * kTile + row < nq;  // padding rows of a ragged tile are not stored
-      const size_t grow = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile + row;
-      uint4* dst = reinterpret_cast<uint4*>(o_ptr + grow * D + (D / 2) * h);
-#pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_row + L::kColO + (D / 2) * h + 32 * c, r);
-        uint32_t pk[16];
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+          if (live) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-        if (live) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int v = 0; v < 4; ++v) dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
         }
+        if (h == 0 && live) lse_ptr[grow] = empty ? -INFINITY : (m_run + lg2(l_tot)) * 0.69314718055994530942f;
       }
-      if (h == 0 && live) lse_ptr[grow] = empty ? -INFINITY : (m_run + lg2(l_tot)) * 0.69314718055994530942f;
+      g += n;
+      ++uu;
     }
   }
 

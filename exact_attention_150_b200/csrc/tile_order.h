@@ -53,4 +53,55 @@ inline int order_group(double bytes_per_problem, int problems) {
   return g < 1.0 ? 1 : static_cast<int>(g);
 }
 
+// Persistent grids: `grid` CTAs share the units (problem, tile) of the
+// launch order above.  The units are dealt in rounds of `grid` items; in
+// round r CTA c takes item r * grid + c for even r and r * grid + grid-1-c
+// for odd r (a snake: the CTA that took the last item of one round takes the
+// first of the next).  Without folding an item is one unit, in launch order.
+// With folding (causal grids, whose tiles get lighter along the order inside
+// a group), item k of a group of S units is the pair of units k and S-1-k of
+// that group: a heavy tile and a light one, so that every item carries about
+// the same work and the CTAs' totals stay within about one item of each
+// other.  Every unit belongs to exactly one item.
+struct UnitPlan {
+  int units;      // problems * tiles
+  int span;       // units of a full group
+  int per_group;  // items of a full group
+  int items;
+  int fold;
+};
+
+ATTN_HD UnitPlan unit_plan(int problems, int tiles, int group, int fold) {
+  UnitPlan p;
+  p.units = problems * tiles;
+  p.span = group * tiles;
+  p.fold = fold;
+  p.per_group = fold ? (p.span + 1) / 2 : p.span;
+  const int full = p.span > 0 ? p.units / p.span : 0;
+  const int tail = p.units - full * p.span;
+  p.items = full * p.per_group + (fold ? (tail + 1) / 2 : tail);
+  return p;
+}
+
+// Unit slots each CTA walks (some of them empty).
+ATTN_HD int unit_slots(const UnitPlan& p, unsigned grid) {
+  const int rounds = static_cast<int>((static_cast<unsigned>(p.items) + grid - 1u) / grid);
+  return p.fold ? 2 * rounds : rounds;
+}
+
+// Unit of slot s of CTA cta, or -1 for an empty slot.
+ATTN_HD int unit_at(const UnitPlan& p, unsigned grid, unsigned cta, int s) {
+  const int r = p.fold ? s >> 1 : s;
+  const unsigned c = (r & 1) ? grid - 1u - cta : cta;
+  const unsigned it = static_cast<unsigned>(r) * grid + c;  // unsigned: may pass 2^31 - 1
+  if (it >= static_cast<unsigned>(p.items)) return -1;
+  if (!p.fold) return static_cast<int>(it);
+  const int g = static_cast<int>(it) / p.per_group;
+  const int k = static_cast<int>(it) - g * p.per_group;
+  const int g0 = g * p.span;
+  const int size = p.units - g0 < p.span ? p.units - g0 : p.span;
+  if ((s & 1) == 0) return g0 + k;
+  return size - 1 - k != k ? g0 + size - 1 - k : -1;
+}
+
 }  // namespace attn
