@@ -431,6 +431,10 @@ def run_ours(args):
         native.backward(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, dq=dq, dk=dk, dv=dv, workspace=ws,
                         phase=phase, deterministic=args.deterministic and phase == native.ATTN_BWD_ALL)
 
+    # The reproducible backward, and every d = 256 backward, is one call of
+    # three kernels (preprocess, dK/dV, dQ) timed as a whole.
+    one_call = args.deterministic or w.d == 256
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
@@ -441,7 +445,7 @@ def run_ours(args):
             return
         if ev is not None:
             ev[1].record(stream)
-        if args.deterministic:
+        if one_call:
             # One call: preprocess, dK/dV and dQ kernels.
             bwd(native.ATTN_BWD_ALL)
             if ev is not None:
@@ -499,11 +503,12 @@ def run_ours(args):
     # Forward algorithmic bytes: read Q, K, V, write O (16-bit) and LSE (fp32).
     fwd_bytes = w.B * w.H * (2 * (2 * w.N + 2 * w.N) * w.d + 4 * w.N)
     kernels = {"fwd_kernel": {"ms": fwd_ms, "tflops": w.fwd_flops() / fwd_ms / 1e9, "gbs": fwd_bytes / fwd_ms / 1e6}}
-    if w.backward and args.deterministic:
+    one_name = ("bwd_deterministic (preprocess, dK/dV and dQ kernels)" if w.d != 256
+                else "bwd, d = 256 (preprocess, 64-key dK/dV and dQ kernels)")
+    if w.backward and one_call:
         det_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-        kernels["bwd_deterministic (preprocess, dK/dV and dQ kernels)"] = {"ms": det_ms,
-                                                                      "tflops": w.bwd_flops() / det_ms / 1e9}
-        dom_name, dom_ms, dom_flops = "bwd_deterministic", det_ms, w.bwd_flops()
+        kernels[one_name] = {"ms": det_ms, "tflops": w.bwd_flops() / det_ms / 1e9}
+        dom_name, dom_ms, dom_flops = one_name.split(" (")[0], det_ms, w.bwd_flops()
     elif w.backward:
         pre_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
         main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -515,14 +520,14 @@ def run_ours(args):
         dom_name, dom_ms, dom_flops = "bwd_main_kernel", main_ms, w.bwd_flops()
     else:
         dom_name, dom_ms, dom_flops = "fwd_kernel", fwd_ms, w.fwd_flops()
-    spans = {"fwd_kernel": (0, 1), "bwd_deterministic (preprocess, dK/dV and dQ kernels)": (1, 2),
+    spans = {"fwd_kernel": (0, 1), one_name: (1, 2),
              "bwd_pre_kernel": (1, 2), "bwd_main_kernel": (2, 3), "bwd_post_kernel": (3, 4)}
     add_spread(kernels, evs, spans)
     for name, kinfo in kernels.items():
         if "tflops" in kinfo:
             kinfo["frac"] = kinfo["tflops"] / peak
     achieved = dom_flops / dom_ms / 1e9
-    traffic = None if args.deterministic else KERNEL_TRAFFIC.get((w.name, w.N), {}).get(dom_name)
+    traffic = None if one_call else KERNEL_TRAFFIC.get((w.name, w.N), {}).get(dom_name)
     if fwd_ms < 0.1:
         ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr())
         code = native.ATTN_BF16 if w.dtype == "bf16" else native.ATTN_FP16

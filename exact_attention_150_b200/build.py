@@ -16,7 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libattn.so")
 SOURCES = [os.path.join(CSRC, "attn_api.cu"), os.path.join(CSRC, "host_step.cpp")]
-HEADERS = [os.path.join(CSRC, f) for f in ("sm100.cuh", "tile_order.h", "trace.h", "fwd_kernel.cuh", "bwd_kernel.cuh", "bwd_dq_kernel.cuh")] + [
+HEADERS = [os.path.join(CSRC, f) for f in ("sm100.cuh", "tile_order.h", "trace.h", "fwd_kernel.cuh", "bwd_kernel.cuh", "bwd_dq_kernel.cuh",
+                                              "bwd_kv_wide_kernel.cuh")] + [
     os.path.join(INCLUDE, "attn.h")]
 
 

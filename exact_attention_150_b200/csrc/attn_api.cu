@@ -14,6 +14,7 @@
 #include "attn.h"
 #include "bwd_dq_kernel.cuh"
 #include "bwd_kernel.cuh"
+#include "bwd_kv_wide_kernel.cuh"
 #include "fwd_kernel.cuh"
 #include "trace.h"
 
@@ -41,16 +42,17 @@ EncodeTiledFn encode_fn() {
 // 3D view [slabs][N][d] of a contiguous 16-bit (or, with e4m3, 8-bit)
 // tensor (a slab is one (batch, head) slice of a dense batch, or one head of
 // a packed variable-length batch), read in boxes 128 bytes wide (64 16-bit
-// or 128 8-bit columns) x 128 rows of one slab, with the 128-byte swizzle
-// the MMA descriptors expect.  Rows past N read as zeros, so a ragged last
-// tile never touches the next slab.
-bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16, bool e4m3 = false) {
+// or 128 8-bit columns) x box_rows rows of one slab, with the 128-byte
+// swizzle the MMA descriptors expect.  Rows past N read as zeros, so a
+// ragged last tile never touches the next slab.
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, bool bf16, bool e4m3 = false,
+              int box_rows = kTile) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t eb = e4m3 ? 1 : 2;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * eb, static_cast<cuuint64_t>(N) * d * eb};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(kTile), 1};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUtensorMapDataType type = e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                         : (bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
@@ -105,6 +107,7 @@ int sm_count() {
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device):
 // the attribute persists, and setting it on every launch costs host time
 // that small problems notice.
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
   static std::mutex mu;
@@ -194,9 +197,11 @@ Problem varlen_problem(int B, int H, int total_q, int total_k, int max_q, int ma
 // Backward workspace of a problem, in 4-byte words: dQ accumulator
 // [(rows + pad) * d] | D [rows] | -log2(e) LSE [rows] | (16-byte aligned)
 // [problems][qtiles] words that no kernel uses at present (they keep the
-// size attn_bwd_workspace_bytes documents), with rows = slabs * rows_q.  The pad takes the reductions of the ragged last
-// query tile's masked rows (exact zeros; see pad_rows); in a packed batch
-// any sequence's last tile can reach up to 127 rows past the total.
+// size attn_bwd_workspace_bytes documents), with rows = slabs * rows_q.
+// The pad takes the reductions of the ragged last query tile's masked rows
+// (exact zeros; see pad_rows); in a packed batch any sequence's last tile
+// can reach up to 127 rows past the total.  The reproducible backward and
+// every d = 256 backward leave the accumulator unused.
 struct WsLayout {
   long long rows, dvec, nlse2, counters, ncounters, words;
 };
@@ -297,6 +302,52 @@ attn_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
 }
 
 
+// The d = 256 backward: preprocess (no accumulator), the dK/dV kernel (one
+// CTA per 64-key tile) and the dQ kernel (one CTA per query tile).  Always
+// reproducible: no kernel adds into memory that another CTA writes.  K and V
+// maps read 64-row boxes.
+template <bool BF16, bool CAUSAL>
+attn_status launch_bwd_wide(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const CUtensorMap& mdo, const void* o, const void* dout, const float* lse, void* dq,
+                            void* dk, void* dv, float* ws, const Problem& pb, float scale, int phase, cudaStream_t st) {
+  constexpr int D = 256;
+  const WsLayout w = ws_layout(pb, D);
+  float* dvec = ws + w.dvec;
+  float* nlse2 = ws + w.nlse2;
+  const float scale_log2 = scale * 1.4426950408889634f;
+  if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_PREPROCESS) {
+    constexpr int kRowsPerBlock = 256 / (D / 8);
+    const long long pre_blocks = (w.rows + kRowsPerBlock - 1) / kRowsPerBlock;
+    attn::bwd_pre_kernel<D, BF16><<<static_cast<unsigned>(pre_blocks), 256, 0, st>>>(
+        static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, dvec, nlse2, nullptr, w.rows);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  if (phase == ATTN_BWD_ALL || phase == ATTN_BWD_MAIN) {
+    using LK = attn::BwdKvWideLayout;
+    auto kk = attn::bwd_kv_wide_kernel<BF16, CAUSAL>;
+    if (set_smem(kk, LK::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
+    // Every CTA of a problem streams its Q and dO rows and their LSE and D.
+    const int gk = attn::order_group((4.0 * D + 8.0) * avg_rows(pb.rows_q, pb), pb.problems);
+    const int ktiles64 = 2 * pb.ktiles;  // 64-key tiles of the longest key sequence, at most
+    const unsigned gridk = static_cast<unsigned>(pb.problems) * static_cast<unsigned>(ktiles64);
+    kk<<<gridk, 384, LK::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, static_cast<uint16_t*>(dk),
+                                       static_cast<uint16_t*>(dv), pb.cu_q, pb.cu_k, pb.H, pb.rows_q, pb.rows_k,
+                                       pb.bottom_right, scale, scale_log2, pb.problems, ktiles64, gk);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    using LQ = attn::BwdDqLayout<D>;
+    auto kq = attn::bwd_dq_kernel<D, BF16, CAUSAL>;
+    if (set_smem(kq, LQ::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
+    // Every CTA of a problem streams its K and V.
+    const int gq = attn::order_group(4.0 * D * avg_rows(pb.rows_k, pb), pb.problems);
+    const unsigned gridq = static_cast<unsigned>(pb.problems) * static_cast<unsigned>(pb.qtiles);
+    kq<<<gridq, 384, LQ::kAlloc, st>>>(mq, mk, mv, mdo, dvec, nlse2, static_cast<uint16_t*>(dq), pb.cu_q, pb.cu_k,
+                                       pb.H, pb.rows_q, pb.rows_k, pb.bottom_right, scale, scale_log2, pb.problems,
+                                       pb.qtiles, gq);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;  // no dQ convert: the dQ kernel writes 16-bit dQ itself
+}
+
 template <int D, bool BF16>
 attn_status dispatch_fwd_causal(int causal, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                 void* o, float* lse, const Problem& pb, float sl2, cudaStream_t st) {
@@ -355,14 +406,23 @@ attn_status dispatch_bwd_causal(int causal, bool det, const CUtensorMap& mq, con
 attn_status bwd_launch(const void* q, const void* k, const void* v, const void* o, const float* lse,
                        const void* dout, void* dq, void* dk, void* dv, void* workspace, const Problem& pb, int d,
                        float scale, int causal, attn_dtype dtype, int phase, bool det, void* stream) {
-  if (d == 256) return ATTN_ERR_UNSUPPORTED;  // see include/attn.h
   const bool bf16 = dtype == ATTN_BF16;
+  const int key_box = d == 256 ? 64 : kTile;  // the d = 256 kernels take 64-key tiles
   CUtensorMap mq, mk, mv, mdo;
-  if (!make_map(&mq, q, pb.slabs, pb.rows_q, d, bf16) || !make_map(&mk, k, pb.slabs, pb.rows_k, d, bf16) ||
-      !make_map(&mv, v, pb.slabs, pb.rows_k, d, bf16) || !make_map(&mdo, dout, pb.slabs, pb.rows_q, d, bf16))
+  if (!make_map(&mq, q, pb.slabs, pb.rows_q, d, bf16) || !make_map(&mk, k, pb.slabs, pb.rows_k, d, bf16, false, key_box) ||
+      !make_map(&mv, v, pb.slabs, pb.rows_k, d, bf16, false, key_box) ||
+      !make_map(&mdo, dout, pb.slabs, pb.rows_q, d, bf16))
     return ATTN_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
+  if (d == 256) {
+    (void)det;  // always reproducible
+#define ATTN_LAUNCH_WIDE(BB, C) \
+  launch_bwd_wide<BB, C>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, pb, scale, phase, st)
+    if (bf16) return causal ? ATTN_LAUNCH_WIDE(true, true) : ATTN_LAUNCH_WIDE(true, false);
+    return causal ? ATTN_LAUNCH_WIDE(false, true) : ATTN_LAUNCH_WIDE(false, false);
+#undef ATTN_LAUNCH_WIDE
+  }
 #define ATTN_DISPATCH_BWD(DD, BB) \
   dispatch_bwd_causal<DD, BB>(causal, det, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, pb, scale, phase, st)
   if (d == 64) return bf16 ? ATTN_DISPATCH_BWD(64, true) : ATTN_DISPATCH_BWD(64, false);
@@ -548,7 +608,6 @@ attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const v
   attn::TraceRange trace("attn_bwd_varlen");
   const attn_status cs = check_varlen(B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
-  if (d == 256) return ATTN_ERR_UNSUPPORTED;  // forward only
   if (B == 0 || H == 0) return ATTN_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (total_q == 0 || max_seqlen_q == 0) {  // no query rows: dK = dV = 0
@@ -609,7 +668,6 @@ attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
   if (phase < ATTN_BWD_ALL || phase > ATTN_BWD_CONVERT) return ATTN_ERR_INVALID_ARG;
   const attn_status cs = check_common(B, H, Nq, Nk, d, causal, dtype);
   if (cs != ATTN_OK) return cs;
-  if (d == 256) return ATTN_ERR_UNSUPPORTED;  // forward only
   if (B == 0 || H == 0) return ATTN_OK;
   if (Nk == 0) return Nq == 0 ? ATTN_OK : ATTN_ERR_INVALID_ARG;
   cudaStream_t st0 = static_cast<cudaStream_t>(stream);

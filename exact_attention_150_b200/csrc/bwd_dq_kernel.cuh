@@ -46,16 +46,26 @@ namespace attn {
 
 template <int D>
 struct BwdDqLayout {
-  static constexpr int kTileRows = 128;
+  static constexpr int kTileRows = 128;                 // query rows of a CTA
+  static constexpr int kKeyRows = D == 256 ? 64 : 128;  // keys of a key tile
+  static constexpr int kKeyHalf = kKeyRows / 2;         // keys of one softmax warpgroup
   static constexpr int kRowBytes = D * 2;
-  static constexpr int kChunks = kRowBytes / 128;      // 128-byte column chunks per row
-  static constexpr int kChunkBytes = kTileRows * 128;  // one 128-row chunk
+  static constexpr int kChunks = kRowBytes / 128;        // 128-byte column chunks per row
+  static constexpr int kChunkBytes = kTileRows * 128;    // one chunk of Q or dO
+  static constexpr int kKeyChunkBytes = kKeyRows * 128;  // one chunk of K or V
   static constexpr int kTileBytes = kTileRows * kRowBytes;
-  static constexpr int kSlots = D == 128 ? 5 : 10;     // K/V ring slots
+  static constexpr int kKeyTileBytes = kKeyRows * kRowBytes;
+  // d = 256: dO stays in shared memory (the A operand of dP has no room in
+  // tensor memory), and once Q has been copied into tensor memory its
+  // staging area serves as two more ring slots.
+  static constexpr bool kWide = D == 256;
+  static constexpr int kSlots = D == 64 ? 10 : 5;       // K/V ring slots
+  static constexpr int kOwnSlots = kWide ? 3 : kSlots;  // slots after dO; the rest alias Q
   static constexpr int kQOff = 0;
   static constexpr int kDOOff = kQOff + kTileBytes;
   static constexpr int kRingOff = kDOOff + kTileBytes;
-  static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kOwnSlots * kKeyTileBytes;
+  static_assert(kWide ? (kSlots - kOwnSlots) * kKeyTileBytes <= kTileBytes : kOwnSlots == kSlots, "ring");
   // qd_full, kv_full[kSlots], kv_empty[kSlots], s_full, s_read, dp_full,
   // ds_full, dq_done, mma_done, qd_tmem
   static constexpr int kNumBars = 1 + 2 * kSlots + 7;
@@ -64,11 +74,11 @@ struct BwdDqLayout {
   static constexpr int kAlloc = kBytes + 1024 <= 232448 ? kBytes + 1024 : 232448;
   static_assert(kBytes <= 232448, "shared memory budget");
   static constexpr uint32_t kColS = 0;
-  static constexpr uint32_t kColDP = 128;
-  static constexpr uint32_t kColDQ = 256;
+  static constexpr uint32_t kColDP = kKeyRows;
+  static constexpr uint32_t kColDQ = 2 * kKeyRows;
   static constexpr uint32_t kColQ = kColDQ + D;      // Q, 16-bit pairs
-  static constexpr uint32_t kColDO = kColQ + D / 2;  // dO, 16-bit pairs
-  static_assert(kColDO + D / 2 <= 512, "tensor memory budget");
+  static constexpr uint32_t kColDO = kColQ + D / 2;  // dO, 16-bit pairs (not at d = 256)
+  static_assert((kWide ? kColQ : kColDO) + D / 2 <= 512, "tensor memory budget");
 };
 
 // dvec and nlse2 hold D_i and -log2(e) LSE_i per query row of the tensor
@@ -83,6 +93,8 @@ __global__ void __launch_bounds__(384, 1)
                   int bottom_right, float scale, float scale_log2, int problems, int grid_tiles, int group) {
   using L = BwdDqLayout<D>;
   constexpr int kT = L::kTileRows;
+  constexpr int kKR = L::kKeyRows;
+  constexpr int kKW = L::kKeyHalf;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -120,7 +132,7 @@ __global__ void __launch_bounds__(384, 1)
     nk = nk < 0 ? 0 : nk;
   }
   const int nqt = (nq + kT - 1) / kT;
-  const int nkt = (nk + kT - 1) / kT;
+  const int nkt = (nk + kKR - 1) / kKR;
   if (ty >= nqt) return;  // a sequence shorter than the grid
   // Causal: the heaviest query tiles are launched first.
   const int qt = CAUSAL ? (nqt - 1 - ty) : ty;
@@ -131,7 +143,7 @@ __global__ void __launch_bounds__(384, 1)
   if (CAUSAL) {
     const int last_row = qt * kT + kT - 1 < nq - 1 ? qt * kT + kT - 1 : nq - 1;
     const int last_key = last_row + off < nk - 1 ? last_row + off : nk - 1;
-    n = last_key < 0 ? 0 : last_key / kT + 1;
+    n = last_key < 0 ? 0 : last_key / kKR + 1;
   }
   const size_t grow0 = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kT;  // first row of the tile
   if (n == 0) {
@@ -174,6 +186,10 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
 
   // Ring items: K_j is item 2j, V_j item 2j + 1 (j < n).
+  auto ring_off = [](int slot) {
+    return slot < L::kOwnSlots ? L::kRingOff + slot * L::kKeyTileBytes
+                               : L::kQOff + (slot - L::kOwnSlots) * L::kKeyTileBytes;
+  };
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -190,15 +206,21 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = true;
       for (; ok && item < 2 * n; ++item) {
         const int slot = item % L::kSlots;
+        // d = 256: the slots in the Q staging area are free once Q is in
+        // tensor memory.
+        if (L::kWide && item == L::kOwnSlots && !mbar_wait(qd_tmem, 0, abort_flag)) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait(&kv_empty[slot], ((item / L::kSlots) & 1) ^ 1, abort_flag)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
-        uint8_t* dst = smem + L::kRingOff + slot * L::kTileBytes;
+        mbar_arrive_expect_tx(&kv_full[slot], L::kKeyTileBytes);
+        uint8_t* dst = smem + ring_off(slot);
         const CUtensorMap* map = (item & 1) ? &tm_v : &tm_k;
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(dst + c * L::kChunkBytes, map, &kv_full[slot], c * 64, k0 + (item >> 1) * kT, z);
+          tma_load_3d(dst + c * L::kKeyChunkBytes, map, &kv_full[slot], c * 64, k0 + (item >> 1) * kKR, z);
       }
       if (!ok) {
         // Let the copies already issued land before the CTA exits.
@@ -209,37 +231,45 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // A (TMEM) x K-major
+    constexpr uint32_t kIdS = idesc_f16(BF16, 128, kKR, false, false);  // A (TMEM or K-major) x K-major
     constexpr uint32_t kIdQ = idesc_f16(BF16, 128, D, false, true);     // dS (TMEM) x K MN-major
-    const uint32_t ring_base = smem_u32(smem + L::kRingOff);
+    const uint32_t smem_base = smem_u32(smem);
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
-    auto slot_addr = [&](int item) { return ring_base + (item % L::kSlots) * L::kTileBytes; };
+    auto slot_addr = [&](int item) { return smem_base + ring_off(item % L::kSlots); };
     auto wait_item = [&](int item) { return wait_all(&kv_full[item % L::kSlots], (item / L::kSlots) & 1); };
-    // B K-major SW128: 32 bytes per K step of 16 inside a 128-byte row, one
-    // 16 KB chunk per 64 columns; A from tensor memory: 8 columns per step.
-    auto kstep = [](int ks) { return static_cast<uint64_t>(((ks >> 2) * L::kChunkBytes + (ks & 3) * 32) >> 4); };
+    // K-major SW128 operands: 32 bytes per K step of 16 inside a 128-byte
+    // row, one chunk per 64 columns (kChunkBytes for the 128-row Q and dO,
+    // kKeyChunkBytes for K and V); A from tensor memory: 8 columns per step.
+    auto kstep_q = [](int ks) { return static_cast<uint64_t>(((ks >> 2) * L::kChunkBytes + (ks & 3) * 32) >> 4); };
+    auto kstep_k = [](int ks) { return static_cast<uint64_t>(((ks >> 2) * L::kKeyChunkBytes + (ks & 3) * 32) >> 4); };
     auto issue_s = [&](int j) {  // S(j) = Q K_j^T
       const uint64_t kd = sdesc_sw128(slot_addr(2 * j), 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
-        mma_ts(tmem + L::kColS, tmem + L::kColQ + 8 * ks, kd + kstep(ks), kIdS, ks > 0 ? 1u : 0u);
+        mma_ts(tmem + L::kColS, tmem + L::kColQ + 8 * ks, kd + kstep_k(ks), kIdS, ks > 0 ? 1u : 0u);
     };
-    auto issue_dp = [&](int j) {  // dP(j) = dO V_j^T
+    auto issue_dp = [&](int j) {  // dP(j) = dO V_j^T (d = 256: dO from shared memory)
       const uint64_t vd = sdesc_sw128(slot_addr(2 * j + 1), 16, 1024);
+      const uint64_t od = sdesc_sw128(smem_base + L::kDOOff, 16, 1024);
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks)
-        mma_ts(tmem + L::kColDP, tmem + L::kColDO + 8 * ks, vd + kstep(ks), kIdS, ks > 0 ? 1u : 0u);
+      for (int ks = 0; ks < D / 16; ++ks) {
+        if constexpr (L::kWide)
+          mma_ss(tmem + L::kColDP, od + kstep_q(ks), vd + kstep_k(ks), kIdS, ks > 0 ? 1u : 0u);
+        else
+          mma_ts(tmem + L::kColDP, tmem + L::kColDO + 8 * ks, vd + kstep_k(ks), kIdS, ks > 0 ? 1u : 0u);
+      }
     };
-    // dQ += dS(j) K_j: A = dS over dP (key step ks of 16 keys: keys
-    // [64h, 64h + 64) sit in columns [64h, 64h + 32), 8 per step), B = K_j
-    // MN-major (16 key rows of 128 bytes per step).
+    // dQ += dS(j) K_j: A = dS over dP (key step ks of 16 keys: the keys
+    // [kKW h, kKW h + kKW) of warpgroup h sit in columns kKW h + [0, kKW/2),
+    // 8 per step), B = K_j MN-major (16 key rows of 128 bytes per step).
     auto issue_dq = [&](int j) {
-      const uint64_t kmn = sdesc_sw128(slot_addr(2 * j), L::kChunkBytes, 1024);
+      const uint64_t kmn = sdesc_sw128(slot_addr(2 * j), L::kKeyChunkBytes, 1024);
+      constexpr int kStepsPerHalf = kKW / 16;
 #pragma unroll
-      for (int ks = 0; ks < kT / 16; ++ks) {
-        const uint32_t ds_col = tmem + L::kColDP + 64 * (ks >> 2) + 8 * (ks & 3);
+      for (int ks = 0; ks < kKR / 16; ++ks) {
+        const uint32_t ds_col = tmem + L::kColDP + kKW * (ks / kStepsPerHalf) + 8 * (ks % kStepsPerHalf);
         mma_ts(tmem + L::kColDQ, ds_col, kmn + 128 * ks, kIdQ, (j > 0 || ks > 0) ? 1u : 0u);
       }
     };
@@ -302,7 +332,24 @@ __global__ void __launch_bounds__(384, 1)
     // head dimension (16-byte units of the 128-byte swizzled tiles) as
     // 32-bit words of two 16-bit values, the lowest index in the low bits.
     bool ok = __all_sync(0xffffffffu, mbar_wait(qd_full, 0, abort_flag));
-    if (ok) {
+    if constexpr (L::kWide) {
+      // d = 256: Q only; each warpgroup copies two whole chunks of its row.
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint8_t* src = smem + L::kQOff + (2 * h + c) * L::kChunkBytes + row * 128;
+          uint32_t w[32];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(src + ((u ^ (row & 7)) * 16));
+            w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
+          }
+          tmem_st32(t_row + L::kColQ + 64 * h + 32 * c, w);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+      }
+    } else if (ok) {
       constexpr bool kTwoChunks = L::kRowBytes == 256;  // each warpgroup copies one whole chunk
       constexpr int kUnits = L::kRowBytes / 32;          // 16-byte units in half a row
 #pragma unroll
@@ -331,17 +378,17 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       // Keys past nk (ragged last tile) and, causal, keys after query + off
       // get P = 0: key column c is kept iff c <= lim.
-      const int kv_valid = nk - j * kT;
-      const int diag_lim = (qt - j) * kT + off;
-      const bool masked = (CAUSAL && diag_lim < kT - 1) || kv_valid < kT;
+      const int kv_valid = nk - j * kKR;
+      const int diag_lim = qt * kT - j * kKR + off;
+      const bool masked = (CAUSAL && diag_lim < kKR - 1) || kv_valid < kKR;
       int lim = kv_valid - 1;
       if (CAUSAL && diag_lim + row < lim) lim = diag_lim + row;
-      float p[64];
+      float p[kKW];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < kKW / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(t_row + L::kColS + 64 * h + 32 * c, r);
-        if (c == 1) {  // S is in registers: S(j+1) may overwrite it
+        tmem_ld32(t_row + L::kColS + kKW * h + 32 * c, r);
+        if (c == kKW / 32 - 1) {  // S is in registers: S(j+1) may overwrite it
           tc_fence_before();
           mbar_arrive(s_read);
         }
@@ -354,20 +401,23 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (masked) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (64 * h + i > lim) p[i] = 0.f;
+        for (int i = 0; i < kKW; ++i)
+          if (kKW * h + i > lim) p[i] = 0.f;
       }
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       // dS = P (dP - D), 16-bit, over dP: keys 2i, 2i + 1 of the warpgroup in
-      // column 128 + 64h + i.  The 64 dP values are loaded first, since the
-      // packed dS lands in the first half of the warpgroup's dP columns.
+      // column kColDP + kKW h + i.  The kKW dP values are loaded first, since
+      // the packed dS lands in the first half of the warpgroup's dP columns.
       const float2 nd2 = make_float2(-dr, -dr);
-      uint32_t r[64];
-      tmem_ld64(t_row + L::kColDP + 64 * h, r);
+      uint32_t r[kKW];
+      if constexpr (kKW == 64)
+        tmem_ld64(t_row + L::kColDP + kKW * h, r);
+      else
+        tmem_ld32(t_row + L::kColDP + kKW * h, r);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < kKW / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -375,7 +425,7 @@ __global__ void __launch_bounds__(384, 1)
           const float2 ds = mul2(make_float2(p[32 * c + 2 * i], p[32 * c + 2 * i + 1]), dpm);
           pk[i] = pack2<BF16>(ds.x, ds.y);
         }
-        tmem_st16(t_row + L::kColDP + 64 * h + 16 * c, pk);
+        tmem_st16(t_row + L::kColDP + kKW * h + 16 * c, pk);
       }
       tmem_st_wait();
       tc_fence_before();

@@ -147,7 +147,7 @@ attn_status attn_host_step(const void* q_h, const void* k_h, const void* v_h, co
   if (causal != ATTN_CAUSAL_NONE && causal != ATTN_CAUSAL_TOP_LEFT && causal != ATTN_CAUSAL_BOTTOM_RIGHT)
     return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_FP16 && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;  // the backward's head dims
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   const long long bh = static_cast<long long>(B) * H;
   if (bh > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if (bh == 0) return ATTN_OK;

@@ -65,13 +65,15 @@ SWEEP = {n: Workload(f"sweep{n}", 4, 32, n, 128, "fp16", False, False, 1003)
          for n in (512, 1024, 2048, 4096, 8192)}
 TRAIN_D64 = Workload("train_d64", 2, 16, 4096, 64, "fp16", True, True, 1004)
 LONG_CTX = Workload("long_ctx", 1, 16, 16384, 128, "bf16", True, True, 1005, 0.5)
-# Head dimension 256 (forward only): the long-context shape at d = 256.
+# Head dimension 256: the long-context shape at d = 256, forward only and
+# forward + backward.
 FWD_D256 = Workload("fwd_d256", 1, 16, 16384, 256, "bf16", True, False, 1006, 0.5)
+LONG_CTX_D256 = Workload("long_ctx_d256", 1, 16, 16384, 256, "bf16", True, True, 1010, 0.5)
 # The long sweep points run causal in bf16: the causal 16-bit forward at
 # N >= 4096, d = 128 on the sweep's batch shape.
 CAUSAL_SWEEP = {n: Workload(f"causal{n}", 4, 32, n, 128, "bf16", True, False, 1008) for n in (4096, 8192)}
 
-ALL = [TINY, LAYER_7B, *SWEEP.values(), TRAIN_D64, LONG_CTX, FWD_D256, *CAUSAL_SWEEP.values()]
+ALL = [TINY, LAYER_7B, *SWEEP.values(), TRAIN_D64, LONG_CTX, FWD_D256, LONG_CTX_D256, *CAUSAL_SWEEP.values()]
 
 
 def by_name(name: str) -> Workload:

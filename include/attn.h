@@ -38,10 +38,9 @@
  *   rows i < Nq - Nk) has an empty softmax: O = 0, LSE = -inf, dQ = 0.
  * LSE.  lse[b][h][i] = ln sum_j exp(scale * q_i . k_j) over the unmasked j:
  *   the natural-log row log-sum-exp of the scaled scores, in fp32.
- * Supported shapes.  d in {64, 128}, and 256 for the forward calls only
- *   (every backward entry point returns ATTN_ERR_UNSUPPORTED for d = 256:
- *   its dV and dK accumulators alone would fill tensor memory); any Nq, Nk >= 0 (the kernels work in
- *   tiles of 128 rows and mask a ragged last tile); causal with any Nq, Nk.
+ * Supported shapes.  d in {64, 128, 256} (the FP8 forward: 128 only); any
+ *   Nq, Nk >= 0 (the kernels work in tiles of 128 rows, or 64 keys for the
+ *   d = 256 backward, and mask a ragged last tile); causal with any Nq, Nk.
  *   The tile counts ceil(Nq / 128) and ceil(Nk / 128) must not exceed 65535,
  *   and B*H and B*H times each tile count must fit in an int (for the packed
  *   calls, with the longest sequence's tile counts); other shapes return
@@ -168,11 +167,13 @@ size_t attn_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d);
  *   workspace    device buffer of attn_bwd_workspace_bytes() bytes, 16-byte
  *                aligned; its contents on entry are ignored and on return are
  *                unspecified.  It must not be shared by calls that overlap.
- * dQ is accumulated with fp32 atomic additions, so its last bits may differ
- * between runs; dK and dV are deterministic.
- * Any finite scale is accepted, 0 and negative ones included.  The kernel
- * adds the per-query terms -LSE_i / scale and -D_i to its fp32 products as
- * pieces of the 16-bit input type; in fp16 they are exact for
+ * For d = 64 and 128 dQ is accumulated with fp32 atomic additions, so its
+ * last bits may differ between runs; dK and dV are deterministic.  For
+ * d = 256 attn_bwd is attn_bwd_deterministic (see there): its dK and dV
+ * accumulators take 64 keys per CTA, and dQ comes from its own kernel.
+ * Any finite scale is accepted, 0 and negative ones included.  At d = 64
+ * and 128 the kernel adds the per-query terms -LSE_i / scale and -D_i to its
+ * fp32 products as pieces of the 16-bit input type; in fp16 they are exact for
  * |LSE_i / scale| < 2^31 and |D_i| < 2^31 (for example any |scale| >= 1e-8
  * with |LSE| <= 20).  Beyond that the call records ATTN_ERR_RANGE in the
  * device status word (attn_last_device_status) and its gradients are not
@@ -196,8 +197,11 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
  * own dQ rows in order; nothing is added atomically, so two calls with the
  * same inputs give identical dQ, dK and dV bits.  The second kernel repeats
  * the S and dP products (7 matrix products per tile pair instead of 5), so
- * it is somewhat slower than attn_bwd.  The dQ accumulator and the order
- * counters of the workspace are not used.  Arguments, workspace and errors
+ * it is somewhat slower than attn_bwd.  At d = 256 the dK/dV kernel takes
+ * 64-key tiles, keeping dV^T and dK^T (two 128-row halves of the head
+ * dimension each) in tensor memory, and the dQ kernel 64-key steps; that is
+ * the only d = 256 backward, which attn_bwd runs as well.  The dQ
+ * accumulator of the workspace is not used.  Arguments, workspace and errors
  * as for attn_bwd.
  */
 attn_status attn_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
@@ -215,6 +219,9 @@ attn_status attn_bwd_deterministic(const void* q, const void* k, const void* v, 
  *   MAIN        recomputes P and accumulates dV, dK (written to dv, dk) and
  *               the fp32 dQ accumulator;
  *   CONVERT     dq = 16-bit(dQ accumulator).
+ * At d = 256 PREPROCESS leaves the accumulator alone, MAIN runs the dK/dV
+ * and dQ kernels of attn_bwd_deterministic (dq written directly) and CONVERT
+ * does nothing.
  * Arguments, validation and errors as for attn_bwd; `phase` outside the
  * enum returns ATTN_ERR_INVALID_ARG.
  */
@@ -282,7 +289,7 @@ size_t attn_bwd_noalloc_max_scratch_bytes(void);
  * continues past the call once every result has reached the host, and the
  * host buffers must stay valid until then.  Host buffers should be
  * page-locked (cudaHostAlloc / pinned); pageable memory works but its
- * copies do not overlap.  d must be 64 or 128.  No query rows (B*H*Nq == 0)
+ * copies do not overlap.  d is 64, 128 or 256.  No query rows (B*H*Nq == 0)
  * writes dK = dV = 0 on the host in stream order; Nq > 0 with Nk = 0
  * returns ATTN_ERR_INVALID_ARG.  An error return may leave part of the work
  * enqueued: synchronize the device before reusing the buffers.  The

@@ -243,16 +243,17 @@ def test_selftest_rejects_null_result(lib):
     assert native.load().attn_selftest_wait_timeout(1000, None, None) == native.ATTN_ERR_INVALID_ARG
 
 
-def test_head_dim_256_is_forward_only(lib):
-    """d = 256 passes the forward's checks (not called here: the pointers are
-    fake) and is refused by every backward entry point before any work."""
-    assert _bwd(d=256) == native.ATTN_ERR_UNSUPPORTED
-    assert _bwd(d=256, Nq=0, dq=None, dout=None, q=None, o=None, lse=None) == native.ATTN_ERR_UNSUPPORTED
-    assert _bwd_varlen(d=256) == native.ATTN_ERR_UNSUPPORTED
-    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, workspace=FAKE,
+def test_head_dim_256_is_validated_like_any_supported_d(lib):
+    """d = 256 passes every entry point's shape checks: a NULL pointer is then
+    what gets refused (nothing is launched with the fake pointers)."""
+    assert _bwd(d=256, q=None) == native.ATTN_ERR_INVALID_ARG
+    assert _bwd(d=256, Nq=0, dq=None, dout=None, q=None, o=None, lse=None, dk=None) == native.ATTN_ERR_INVALID_ARG
+    assert _bwd_varlen(d=256, q=None) == native.ATTN_ERR_INVALID_ARG
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, workspace=None,
                 B=1, H=1, Nq=128, Nk=128, d=256, scale=0.1, causal=0, dtype=native.ATTN_BF16, stream=None)
-    assert native.attn_bwd_deterministic(**args) == native.ATTN_ERR_UNSUPPORTED
-    assert _fwd(d=256, q=None) == native.ATTN_ERR_INVALID_ARG  # validated like any supported d
+    assert native.attn_bwd_deterministic(**args) == native.ATTN_ERR_INVALID_ARG
+    assert _fwd(d=256, q=None) == native.ATTN_ERR_INVALID_ARG
+    assert _bwd(d=96, q=None) == native.ATTN_ERR_UNSUPPORTED
 
 
 def _fwd_fp8(**kw):
@@ -318,8 +319,9 @@ def test_host_step_device_bytes_empty(lib):
 
 def test_host_step_validation(lib):
     assert _host_step(chunks=0) == native.ATTN_ERR_INVALID_ARG
-    for d in (256, 96, 0):
+    for d in (96, 0):
         assert _host_step(d=d) == native.ATTN_ERR_UNSUPPORTED
+    assert _host_step(d=256, q=None) == native.ATTN_ERR_INVALID_ARG  # a supported d: checked further
     assert _host_step(dtype=5) == native.ATTN_ERR_UNSUPPORTED
     assert _host_step(causal=3) == native.ATTN_ERR_INVALID_ARG
     for field in ("B", "H", "Nq", "Nk"):

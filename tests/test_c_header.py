@@ -31,7 +31,9 @@ int main(void) {
   EXPECT(attn_fwd(p, p, p, p, (float*)p, 1, 1, 128, 128, 64, 0.125f, 7, ATTN_BF16, NULL) == ATTN_ERR_INVALID_ARG);
   EXPECT(attn_fwd(NULL, NULL, NULL, NULL, NULL, 0, 1, 128, 128, 64, 0.125f, ATTN_CAUSAL_TOP_LEFT, ATTN_FP16, NULL)
          == ATTN_OK);
-  EXPECT(attn_bwd(p, p, p, p, (const float*)p, p, p, p, p, p, 1, 1, 128, 128, 256, 0.1f,
+  EXPECT(attn_bwd(p, p, p, p, (const float*)p, p, p, p, p, NULL, 1, 1, 128, 128, 256, 0.1f,
+                  ATTN_CAUSAL_BOTTOM_RIGHT, ATTN_BF16, NULL) == ATTN_ERR_INVALID_ARG);
+  EXPECT(attn_bwd(p, p, p, p, (const float*)p, p, p, p, p, p, 1, 1, 128, 128, 96, 0.1f,
                   ATTN_CAUSAL_BOTTOM_RIGHT, ATTN_BF16, NULL) == ATTN_ERR_UNSUPPORTED);
   EXPECT(attn_bwd_deterministic(p, p, p, p, (const float*)p, p, NULL, p, p, p, 1, 1, 128, 128, 64, 0.1f,
                                 ATTN_CAUSAL_NONE, ATTN_FP16, NULL) == ATTN_ERR_INVALID_ARG);
@@ -41,8 +43,8 @@ int main(void) {
   EXPECT(attn_bwd_workspace_bytes(0, 1, 128, 128, 64) == 0);
   EXPECT(attn_fwd_varlen(p, p, p, p, (float*)p, NULL, cu, 2, 1, 300, 300, 200, 200, 64, 0.1f,
                          ATTN_CAUSAL_TOP_LEFT, ATTN_BF16, NULL) == ATTN_ERR_INVALID_ARG);
-  EXPECT(attn_bwd_varlen(p, p, p, p, (const float*)p, p, p, p, p, p, cu, cu, 2, 1, 300, 300, 200, 200, 256, 0.1f,
-                         ATTN_CAUSAL_NONE, ATTN_BF16, 0, NULL) == ATTN_ERR_UNSUPPORTED);
+  EXPECT(attn_bwd_varlen(p, p, p, p, (const float*)p, p, p, p, p, p, NULL, cu, 2, 1, 300, 300, 200, 200, 256, 0.1f,
+                         ATTN_CAUSAL_NONE, ATTN_BF16, 0, NULL) == ATTN_ERR_INVALID_ARG);
   EXPECT(attn_bwd_varlen_workspace_bytes(2, 1, 300, 200, 64) > 0);
   EXPECT(attn_fwd_fp8(p, p, p, p, (float*)p, 1, 1, 128, 128, 64, 0.1f, 1.f, 1.f, 1.f, ATTN_CAUSAL_NONE, NULL)
          == ATTN_ERR_UNSUPPORTED);

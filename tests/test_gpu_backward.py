@@ -97,6 +97,62 @@ def test_backward_bottom_right_d64_fp16():
     check_grads_all_slices(q, k, v, do, "bottom_right", 0.125, "bottom-right d64 fp16")
 
 
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n", [1, 64, 100, 300, 640])
+def test_backward_d256(dtype, causal, n):
+    """Head dimension 256: the 64-key dK/dV kernel and the dQ kernel with
+    64-key steps, one to several tiles with a ragged tail."""
+    q, k, v, do = draw(1, 2, n, n, 256, dtype, seed=900 + n, with_grad=True)
+    check_grads_all_slices(q, k, v, do, causal, 1 / 16, f"d256 N{n} {dtype} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True, "bottom_right"])
+@pytest.mark.parametrize("nq,nk", [(100, 300), (300, 100), (1, 257), (257, 1), (200, 640), (640, 64)])
+def test_backward_d256_nq_ne_nk(causal, nq, nk):
+    """Includes key tiles that no query sees (causal with Nk > Nq) and query
+    rows that see no key (bottom-right with Nq > Nk)."""
+    q, k, v, do = draw(2, 2, nq, nk, 256, torch.bfloat16, seed=951 + nq + nk, with_grad=True)
+    check_grads_all_slices(q, k, v, do, causal, 1 / 16, f"d256 Nq{nq} Nk{nk} causal={causal}")
+
+
+def test_backward_d256_long_causal_one_slice():
+    """Several query and key tiles per CTA: B1 H1 N1536 causal bf16 against
+    the full oracle."""
+    q, k, v, do = draw(1, 1, 1536, 1536, 256, torch.bfloat16, seed=961, with_grad=True)
+    check_grads_all_slices(q, k, v, do, True, 1 / 16, "d256 N1536 causal")
+
+
+def test_backward_d256_is_reproducible_and_deterministic_mode_agrees():
+    """The d = 256 backward has no atomics: repeated calls, and
+    attn_bwd against attn_bwd_deterministic, give identical bits."""
+    q, k, v, do = (t.to(DEV) for t in draw(2, 3, 700, 700, 256, torch.bfloat16, seed=971, with_grad=True))
+    o, lse = native.forward(q, k, v, causal=True)
+    a = native.backward(q, k, v, o, lse, do, causal=True)
+    b = native.backward(q, k, v, o, lse, do, causal=True)
+    c = native.backward(q, k, v, o, lse, do, causal=True, deterministic=True)
+    torch.cuda.synchronize()
+    native.device_status()
+    for x, y, z in zip(a, b, c):
+        assert torch.equal(x, y) and torch.equal(x, z)
+
+
+def test_backward_d256_phases_compose():
+    """attn_bwd_phase at d = 256: PREPROCESS then MAIN (which writes dq
+    itself) then CONVERT (nothing) gives attn_bwd's bits."""
+    q, k, v, do = (t.to(DEV) for t in draw(1, 2, 384, 384, 256, torch.float16, seed=981, with_grad=True))
+    o, lse = native.forward(q, k, v)
+    ref = native.backward(q, k, v, o, lse, do)
+    ws = torch.empty(native.attn_bwd_workspace_bytes(1, 2, 384, 384, 256), dtype=torch.uint8, device=DEV)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for ph in (native.ATTN_BWD_PREPROCESS, native.ATTN_BWD_MAIN, native.ATTN_BWD_CONVERT):
+        native.backward(q, k, v, o, lse, do, dq=dq, dk=dk, dv=dv, workspace=ws, phase=ph)
+    torch.cuda.synchronize()
+    native.device_status()
+    for x, y in zip(ref, (dq, dk, dv)):
+        assert torch.equal(x, y)
+
+
 def test_backward_no_queries_gives_zero_dk_dv():
     q = torch.zeros(1, 2, 0, 64, dtype=torch.float16, device=DEV)
     k = torch.randn(1, 2, 130, 64, device=DEV).half()

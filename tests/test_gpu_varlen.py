@@ -74,7 +74,8 @@ def check_against_oracle(inputs, outputs, causal, d, dtype, tag):
 
 
 @pytest.mark.parametrize("causal", [False, True, "bottom_right"])
-@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float16, 64)])
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float16, 64), (torch.bfloat16, 256),
+                                     (torch.float16, 256)])
 def test_varlen_self_attention(causal, dtype, d):
     lens = [1, 130, 0, 257, 64, 500]
     inputs, outputs = run(lens, lens, 2, d, dtype, causal, seed=801)
@@ -82,17 +83,19 @@ def test_varlen_self_attention(causal, dtype, d):
 
 
 @pytest.mark.parametrize("causal", [False, True, "bottom_right"])
-def test_varlen_cross_lengths(causal):
+@pytest.mark.parametrize("d", [64, 256])
+def test_varlen_cross_lengths(causal, d):
     """Different query and key lengths per sequence, including a sequence
     with queries and no keys and one with keys and no queries."""
     lens_q = [100, 3, 300, 0, 50]
     lens_k = [200, 50, 1, 70, 0]
-    inputs, outputs = run(lens_q, lens_k, 3, 64, torch.bfloat16, causal, seed=811)
-    check_against_oracle(inputs, outputs, causal, 64, torch.bfloat16, f"varlen cross causal={causal}")
+    inputs, outputs = run(lens_q, lens_k, 3, d, torch.bfloat16, causal, seed=811)
+    check_against_oracle(inputs, outputs, causal, d, torch.bfloat16, f"varlen cross d{d} causal={causal}")
 
 
-def test_varlen_equal_lengths_match_dense_bitwise():
-    B, H, N, d = 3, 2, 384, 128
+@pytest.mark.parametrize("d", [128, 256])
+def test_varlen_equal_lengths_match_dense_bitwise(d):
+    B, H, N = 3, 2, 384
     q, k, v, do = draw(B, H, N, N, d, torch.bfloat16, seed=821, with_grad=True)
     dev = [t.to(DEV) for t in (q, k, v, do)]
     o, lse = native.forward(*dev[:3], causal=True)
