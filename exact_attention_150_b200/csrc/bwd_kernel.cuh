@@ -14,7 +14,7 @@
 //                       P^T   = exp2(S'^T * scale * log2e)
 //                       dS^T  = P^T * dP'^T
 //                       dV_j += P^T dO_i              (A = P^T from TMEM)
-//                       dK_j += dS^T Q_i              (A = dS^T from shared memory)
+//                       dK_j += dS^T Q_i              (A = dS^T from TMEM)
 //                       dQacc_i += scale * dS K_j     (fp32 atomics)
 //                     then dK_j = scale * dK_j and dV_j are written once.
 //                     (dQ is formed transposed, dQ^T = K_j^T dS^T, when
@@ -32,17 +32,21 @@
 // Tensor memory (d = 128):
 //   [0,128)    S^T fp32; overwritten in place by P^T (16-bit pairs) in
 //              [0,32) and [64,96)
-//   [128,256)  dP^T fp32, then dQ^T = K^T dS^T fp32 (lane = head-dim index)
+//   [128,256)  dP^T fp32, then dS^T packed 16-bit over it, then
+//              dQ^T = K^T dS^T fp32 (lane = head-dim index)
 //   [256,384)  dV,  [384,512) dK
 // For d = 64 the dQ tile is dS K (lane = query row) in [128,192), dV in
 // [256,320) and dK in [320,384).
-// dS^T lives only in shared memory (128-byte swizzled, [key][query]): it is
-// the K-major A operand of dK += dS^T Q and an MN-major operand of the dQ
-// product.  Keeping it out of TMEM lets the next query tile's S^T be issued
-// right after dV, so per query tile the MMA issue order is
+// The dS pass writes dS^T twice: packed 16-bit over dP^T in TMEM, the A
+// operand of dK += dS^T Q (a TS product, which reads only Q from shared
+// memory), and 128-byte swizzled into shared memory ([key][query]), the
+// MN-major operand of the dQ product, which then overwrites the dP^T
+// columns (the tensor core runs dK first).  S^T lives in its own columns,
+// so the next query tile's S^T is issued right after dV, and per query tile
+// the MMA issue order is
 //   dP^T, dV, S^T(next), dK, dQ
-// and the softmax warps go from this tile's dS pass straight to the next
-// tile's P pass while dK and dQ run on the tensor core.
+// while the softmax warps go from this tile's dS pass straight to the next
+// tile's P pass as dK and dQ run on the tensor core.
 // The per-query terms -LSE_i / scale and -D_i enter through one extra K step
 // of 16 in the S^T and dP^T products: the A operand is a constant tile that
 // selects them ([w0,w1,w2,w3,0,...] or [0,0,0,0,w0,w1,w2,w3,0,...] in every
@@ -374,7 +378,6 @@ __global__ void __launch_bounds__(512, 1)
     // and 16 KB per 64-column chunk; MN-major ones step 16 rows (2048 bytes).
     auto kmaj = [](int ks) { return static_cast<uint64_t>(((ks >> 2) * L::kChunkBytes + (ks & 3) * 32) >> 4); };
     const uint64_t kd_k = sdesc_sw128(k_addr, 16, 1024), kd_v = sdesc_sw128(v_addr, 16, 1024);
-    const uint64_t kd_ds = sdesc_sw128(ds_addr, 16, 1024);
     const uint64_t mn_k = sdesc_sw128(k_addr, L::kChunkBytes, 1024), mn_ds = sdesc_sw128(ds_addr, L::kChunkBytes, 1024);
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
@@ -459,14 +462,11 @@ __global__ void __launch_bounds__(512, 1)
       if (!(ok = wait_all(ds_full, it & 1))) break;
       tc_fence_after();
       if (elect_one()) {
-        // dK += dS^T Q: A = dS^T (DQ: K-major in shared memory; otherwise
-        // packed over dP^T in tensor memory), B = Q MN-major.
+        // dK += dS^T Q: A = dS^T packed over dP^T in tensor memory, B = Q
+        // MN-major.
 #pragma unroll
         for (int ks = 0; ks < kBwdTile / 16; ++ks) {
-          if constexpr (DQ)
-            mma_ss(tmem + kColDK, kd_ds + kmaj(ks), qd_mn + 128 * ks, kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
-          else
-            mma_ts(tmem + kColDK, tmem + kColDP + p_col(ks), qd_mn + 128 * ks, kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tmem + kColDK, tmem + kColDP + p_col(ks), qd_mn + 128 * ks, kIdAcc, (it > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(&qd_empty[it % L::kStages]);
         if (it == n_it - 1) mma_commit(acc_full);
@@ -586,11 +586,11 @@ __global__ void __launch_bounds__(512, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
-      // dS pass: dS^T = P^T * dP'^T, packed 16-bit.  DQ: into the 128-byte-
-      // swizzled shared tile (row r, 64 queries per 16 KB chunk), the
-      // operand of both dK and dQ.  Otherwise over dP^T in tensor memory,
-      // in the column layout of P^T (queries 2i, 2i + 1 of chunk c in
-      // column 64h + 16c + i), each chunk landing in columns already read.
+      // dS pass: dS^T = P^T * dP'^T, packed 16-bit, over dP^T in tensor
+      // memory in the column layout of P^T (queries 2i, 2i + 1 of chunk c in
+      // column 64h + 16c + i, each chunk landing in columns already read):
+      // the A operand of dK.  DQ: also into the 128-byte-swizzled shared
+      // tile (row r, 64 queries per 16 KB chunk), the operand of dQ.
       if (!__all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag))) break;
       tc_fence_after();
 #pragma unroll
@@ -616,15 +616,11 @@ __global__ void __launch_bounds__(512, 1)
             }
           }
         }
-        if constexpr (!DQ) tmem_st16(t_row + kColDP + 64 * h + 16 * c, dsk);
+        tmem_st16(t_row + kColDP + 64 * h + 16 * c, dsk);
       }
-      if constexpr (DQ) {
-        tc_fence_before();
-        fence_proxy_async_smem();
-      } else {
-        tmem_st_wait();
-        tc_fence_before();
-      }
+      tmem_st_wait();
+      tc_fence_before();
+      if constexpr (DQ) fence_proxy_async_smem();
       mbar_arrive(ds_full);
     }
   } else if (warp >= 12) {
