@@ -219,8 +219,9 @@ WsLayout ws_layout(const Problem& pb, int d) {
 }
 
 template <int D, bool BF16, bool CAUSAL, bool F8 = false>
-attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse,
-                       const Problem& pb, float scale_log2, cudaStream_t st, float o_scale = 1.f) {
+attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                       void* o, float* lse, const Problem& pb, float scale_log2, cudaStream_t st,
+                       float o_scale = 1.f) {
   using L = attn::FwdLayout<D, F8>;
   auto kern = attn::fwd_kernel<D, BF16, CAUSAL, F8>;
   if (set_smem(kern, L::kAlloc) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -235,7 +236,7 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   // Causal grids with at least two units per CTA deal heavy and light tiles
   // out in pairs (tile_order.h).
   const int fold = CAUSAL && units >= 2u * sms ? 1 : 0;
-  kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, static_cast<uint16_t*>(o), lse, pb.cu_q, pb.cu_k, pb.H, pb.rows_q,
+  kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, mo, static_cast<uint16_t*>(o), lse, pb.cu_q, pb.cu_k, pb.H, pb.rows_q,
                                      pb.rows_k, pb.bottom_right, scale_log2, pb.problems, pb.qtiles, group, fold,
                                      o_scale);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -350,44 +351,46 @@ attn_status launch_bwd_wide(const CUtensorMap& mq, const CUtensorMap& mk, const 
 
 template <int D, bool BF16>
 attn_status dispatch_fwd_causal(int causal, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                                void* o, float* lse, const Problem& pb, float sl2, cudaStream_t st) {
-  return causal ? launch_fwd<D, BF16, true>(mq, mk, mv, o, lse, pb, sl2, st)
-                : launch_fwd<D, BF16, false>(mq, mk, mv, o, lse, pb, sl2, st);
+                                const CUtensorMap& mo, void* o, float* lse, const Problem& pb, float sl2,
+                                cudaStream_t st) {
+  return causal ? launch_fwd<D, BF16, true>(mq, mk, mv, mo, o, lse, pb, sl2, st)
+                : launch_fwd<D, BF16, false>(mq, mk, mv, mo, o, lse, pb, sl2, st);
 }
 
 // The forward launch shared by attn_fwd and attn_fwd_varlen.
 attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const Problem& pb, int d,
                      float scale, int causal, attn_dtype dtype, void* stream) {
   const bool bf16 = dtype == ATTN_BF16;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, q, pb.slabs, pb.rows_q, d, bf16) || !make_map(&mk, k, pb.slabs, pb.rows_k, d, bf16) ||
-      !make_map(&mv, v, pb.slabs, pb.rows_k, d, bf16))
+      !make_map(&mv, v, pb.slabs, pb.rows_k, d, bf16) || !make_map(&mo, o, pb.slabs, pb.rows_q, d, bf16))
     return ATTN_ERR_CUDA;
   const float sl2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 64)
-    return bf16 ? dispatch_fwd_causal<64, true>(causal, mq, mk, mv, o, lse, pb, sl2, st)
-                : dispatch_fwd_causal<64, false>(causal, mq, mk, mv, o, lse, pb, sl2, st);
+    return bf16 ? dispatch_fwd_causal<64, true>(causal, mq, mk, mv, mo, o, lse, pb, sl2, st)
+                : dispatch_fwd_causal<64, false>(causal, mq, mk, mv, mo, o, lse, pb, sl2, st);
   if (d == 256)
-    return bf16 ? dispatch_fwd_causal<256, true>(causal, mq, mk, mv, o, lse, pb, sl2, st)
-                : dispatch_fwd_causal<256, false>(causal, mq, mk, mv, o, lse, pb, sl2, st);
-  return bf16 ? dispatch_fwd_causal<128, true>(causal, mq, mk, mv, o, lse, pb, sl2, st)
-              : dispatch_fwd_causal<128, false>(causal, mq, mk, mv, o, lse, pb, sl2, st);
+    return bf16 ? dispatch_fwd_causal<256, true>(causal, mq, mk, mv, mo, o, lse, pb, sl2, st)
+                : dispatch_fwd_causal<256, false>(causal, mq, mk, mv, mo, o, lse, pb, sl2, st);
+  return bf16 ? dispatch_fwd_causal<128, true>(causal, mq, mk, mv, mo, o, lse, pb, sl2, st)
+              : dispatch_fwd_causal<128, false>(causal, mq, mk, mv, mo, o, lse, pb, sl2, st);
 }
 
 // The FP8 forward launch shared by attn_fwd_fp8 and attn_fwd_fp8_varlen (d = 128).
 attn_status fwd_fp8_impl(const void* q, const void* k, const void* v, void* o, float* lse, const Problem& pb,
                          float scale, float descale_q, float descale_k, float descale_v, int causal, void* stream) {
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, q, pb.slabs, pb.rows_q, 128, true, true) ||
       !make_map(&mk, k, pb.slabs, pb.rows_k, 128, true, true) ||
-      !make_map(&mv, v, pb.slabs, pb.rows_k, 128, true, true))
+      !make_map(&mv, v, pb.slabs, pb.rows_k, 128, true, true) ||
+      !make_map(&mo, o, pb.slabs, pb.rows_q, 128, true))  // O is bf16
     return ATTN_ERR_CUDA;
   // The scores are scale * (descale_q q) . (descale_k k): one factor, in log2 units.
   const float sl2 = scale * descale_q * descale_k * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return causal ? launch_fwd<128, true, true, true>(mq, mk, mv, o, lse, pb, sl2, st, descale_v)
-                : launch_fwd<128, true, false, true>(mq, mk, mv, o, lse, pb, sl2, st, descale_v);
+  return causal ? launch_fwd<128, true, true, true>(mq, mk, mv, mo, o, lse, pb, sl2, st, descale_v)
+                : launch_fwd<128, true, false, true>(mq, mk, mv, mo, o, lse, pb, sl2, st, descale_v);
 }
 
 template <int D, bool BF16>

@@ -64,12 +64,19 @@ struct FwdLayout {
   static constexpr int kTileBytes = kTile * kRowBytes;    // one 128 x D tile
   static constexpr int kKeysPerStep = 32 / kElemBytes;    // keys per MMA K step (32 bytes)
   static constexpr bool kWide = D == 256;                 // see below
-  static constexpr int kSlots = kWide ? 2 : (kTileBytes == 32768 ? 5 : 10);  // K/V ring slots
+  static constexpr int kSlots = kWide ? 2 : (kTileBytes == 32768 ? 4 : 10);  // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kTileBytes;
+  // d <= 128: the epilogue stages the 16-bit O tile here (128-byte
+  // swizzled chunks of 64 columns, the layout of a TMA load) and writes it
+  // with TMA stores.  d = 256 has no room and stores from registers.
+  static constexpr bool kStageO = !kWide;
+  static constexpr int kOChunks = D * 2 / 128 > 0 ? D * 2 / 128 : 1;
+  static constexpr int kOOff = kRingOff + kSlots * kTileBytes;
+  static constexpr int kOBytes = kStageO ? kTile * D * 2 : 0;
   // Exchange between the two softmax warpgroups: row maxima
   // [2 parity][2 warpgroups][128 rows], then row sums [2][2][128].
-  static constexpr int kXOff = kRingOff + kSlots * kTileBytes;
+  static constexpr int kXOff = kOOff + kOBytes;
   static constexpr int kXBytes = 2 * 2 * 2 * kTile * 4;
   // 128 x 16 tile of ones (unswizzled K-major core matrices): B operand of
   // the row-sum product L += P 1.
@@ -77,8 +84,8 @@ struct FwdLayout {
   static constexpr int kOnesBytes = kTile * 16 * 2;
   static constexpr int kBarOff = kOnesOff + kOnesBytes;
   // q_full, q_tmem, kv_full[kSlots], kv_empty[kSlots], s_full[2], p_full[2], pv_done, o_full, mma_done,
-  // xmax[2], xsum
-  static constexpr int kNumBars = 2 + 2 * kSlots + 10;
+  // xmax[2], xsum, o_free, o_staged
+  static constexpr int kNumBars = 2 + 2 * kSlots + 12;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024 <= 232448 ? kBytes + 1024 : 232448;
@@ -103,7 +110,8 @@ struct FwdLayout {
 template <int D, bool BF16, bool CAUSAL, bool F8 = false>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o_ptr,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               uint16_t* __restrict__ o_ptr,
                float* __restrict__ lse_ptr, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H,
                int Nq, int Nk, int bottom_right, float scale_log2, int problems, int grid_tiles, int group,
                int fold, float o_scale) {
@@ -124,6 +132,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* mma_done = o_full + 1;
   uint64_t* xmax_bar = mma_done + 1;  // [2], 256 arrivals each
   uint64_t* xsum_bar = xmax_bar + 2;  // 256 arrivals
+  uint64_t* o_free = xsum_bar + 1;    // the O staging tile may be written (thread 128 arrives)
+  uint64_t* o_staged = o_free + 1;    // 256 arrivals: the O tile is staged
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   float* xchg = reinterpret_cast<float*>(smem + L::kXOff);                 // [2 parity][2 wg][128]
@@ -210,6 +220,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&xmax_bar[0], 256);
     mbar_init(&xmax_bar[1], 256);
     mbar_init(xsum_bar, 256);
+    mbar_init(o_free, 1);
+    mbar_init(o_staged, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -407,6 +419,7 @@ __global__ void __launch_bounds__(384, 1)
     const bool pos_scale = scale_log2 > 0.f;
     const float cx = pos_scale ? scale_log2 : 1.f;
     int uu = 0, g = 0;  // units with key tiles, key tiles before the current unit
+    int ot = 0;         // O tiles staged so far
     bool ok = true;
     for (int r = 0; ok && r < slots; ++r) {
       const int u = unit_index(r);
@@ -618,25 +631,62 @@ __global__ void __launch_bounds__(384, 1)
         const float inv = empty ? 0.f : (F8 ? o_scale : 1.f) / l_tc;
         const bool live = qt * kTile + row < nq;  // padding rows of a ragged tile are not stored
         const size_t grow = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile + row;
+        // O leaves through the staging tile and TMA stores (rows past the
+        // map's extent are not written) for dense batches and for full tiles
+        // of packed ones; a ragged tile of a packed batch stores its live rows
+        // from registers, so that it never touches the next sequence's rows.
+        // Thread 128 issues the stores; it lets the tile be rewritten once
+        // its previous stores have read it (o_free), and stores it once
+        // every softmax thread has staged its part (o_staged).
+        const bool staged = L::kStageO && (cu_q == nullptr || qt * kTile + kTile <= nq);
+        if (staged) {
+          if (threadIdx.x == 128) {
+            tma_store_wait_read();
+            mbar_arrive(o_free);
+          }
+          ok = __all_sync(0xffffffffu, mbar_wait(o_free, ot & 1, abort_flag));
+        }
         uint4* dst = reinterpret_cast<uint4*>(o_ptr + grow * D + (D / 2) * h);
 #pragma unroll 1
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; ok && c < D / 64; ++c) {
           uint32_t r[32];
           tmem_ld32(t_row + L::kColO + (D / 2) * h + 32 * c, r);
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             pk[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-          if (live) {
+          if (staged) {
+            // 16-byte unit u of the row (columns 8u .. 8u+7) sits in chunk
+            // u / 8 at swizzled position (u % 8) ^ (row % 8).
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int u = D * h / 16 + 4 * c + v;
+              *reinterpret_cast<uint4*>(smem + L::kOOff + (u / 8) * L::kChunkBytes + row * 128 +
+                                        (((u % 8) ^ (row & 7)) * 16)) =
+                  make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          } else if (live) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           }
+        }
+        if (staged) {
+          fence_proxy_async_smem();
+          mbar_arrive(o_staged);
+          if (threadIdx.x == 128 && mbar_wait(o_staged, ot & 1, abort_flag)) {
+            for (int c = 0; c < L::kOChunks; ++c)
+              tma_store_3d(&tm_o, smem + L::kOOff + c * L::kChunkBytes, c * 64, q0 + qt * kTile, z);
+            tma_store_commit();
+          }
+          ++ot;
         }
         if (h == 0 && live) lse_ptr[grow] = empty ? -INFINITY : (m_run + lg2(l_tot)) * 0.69314718055994530942f;
       }
       g += n;
       ++uu;
     }
+    // The last O stores have landed before the CTA (and its shared memory) ends.
+    if (threadIdx.x == 128) tma_store_wait_all();
   }
 
   tc_fence_before();

@@ -134,6 +134,23 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// 3D tiled store of box (x, y, z) of `map` from shared memory (the layout
+// tma_load_3d writes); rows of y past the extent of the map are not
+// written.  x must be a multiple of 16 bytes' worth of elements and x, y, z
+// must not be negative.  The issuing thread tracks completion through bulk
+// groups: tma_store_commit closes one, tma_store_wait_read waits until
+// every closed group has finished reading shared memory, tma_store_wait_all
+// until every one has been written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Dynamic shared memory actually granted to this CTA, in bytes.
 __device__ __forceinline__ uint32_t dynamic_smem_bytes() {
   uint32_t v;
