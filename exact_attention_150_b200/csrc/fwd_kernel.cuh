@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(384, 1)
                uint16_t* __restrict__ o_ptr,
                float* __restrict__ lse_ptr, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H,
                int Nq, int Nk, int bottom_right, float scale_log2, int problems, int grid_tiles, int group,
-               int fold, float o_scale) {
+               int fold, int early_q, float o_scale) {
   static_assert(!F8 || BF16, "the 8-bit forward writes bf16");
   using L = FwdLayout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
@@ -420,30 +420,14 @@ __global__ void __launch_bounds__(384, 1)
     const float cx = pos_scale ? scale_log2 : 1.f;
     int uu = 0, g = 0;  // units with key tiles, key tiles before the current unit
     int ot = 0;         // O tiles staged so far
-    bool ok = true;
-    for (int r = 0; ok && r < slots; ++r) {
-      const int u = unit_index(r);
-      if (u < 0) continue;
-      const Unit w = unit_of(u);
-      if (!w.live) continue;
-      const int z = w.z, q0 = w.q0, nq = w.nq, nk = w.nk, qt = w.qt, n = w.n, off = w.off;
-      if (n == 0) {
-        // No row of this tile sees a key (bottom-right with nq > nk, or a
-        // sequence without keys): the softmax is empty, O = 0 and LSE = log 0.
-        const int rows = nq - qt * kTile < kTile ? nq - qt * kTile : kTile;
-        const size_t grow0 = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile;
-        const int t0 = static_cast<int>(threadIdx.x) - 128;  // the 256 softmax threads
-        for (int e = t0; e < rows * D / 8; e += 256)
-          reinterpret_cast<uint4*>(o_ptr + grow0 * D)[e] = make_uint4(0u, 0u, 0u, 0u);
-        for (int e = t0; e < rows; e += 256) lse_ptr[grow0 + e] = -INFINITY;
-        continue;
-      }
-      // Q -> TMEM: this thread copies its row's half of the head dimension
-      // (16-byte units of the 128-byte swizzled tile) as 32-bit words of two
-      // 16-bit or four 8-bit values, the lowest K index in the lowest bits.
-      ok = __all_sync(0xffffffffu, mbar_wait(q_full, uu & 1, abort_flag));
-      if constexpr (!L::kWide) {  // d = 256: Q stays in shared memory
-        if (ok) {
+    // Q -> TMEM: this thread copies its row's half of the head dimension
+    // (16-byte units of the 128-byte swizzled tile) as 32-bit words of two
+    // 16-bit or four 8-bit values, the lowest K index in the lowest bits
+    // (d = 256: Q stays in shared memory; only the handshake remains).
+    auto copy_q = [&](uint32_t parity) {
+      const bool landed = __all_sync(0xffffffffu, mbar_wait(q_full, parity, abort_flag));
+      if constexpr (!L::kWide) {
+        if (landed) {
           constexpr bool kTwoChunks = L::kRowBytes == 256;  // each warpgroup copies one whole chunk
           constexpr int kUnits = L::kRowBytes / 32;          // 16-byte units in half a row
           const uint8_t* qrow = smem + L::kQOff + (kTwoChunks ? h * L::kChunkBytes : 0) + row * 128;
@@ -463,8 +447,30 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_before();
         }
       }
-
       mbar_arrive(q_tmem);
+      return landed;
+    };
+    bool q_ready = false;  // the next unit's Q is already in tensor memory
+    bool ok = true;
+    for (int r = 0; ok && r < slots; ++r) {
+      const int u = unit_index(r);
+      if (u < 0) continue;
+      const Unit w = unit_of(u);
+      if (!w.live) continue;
+      const int z = w.z, q0 = w.q0, nq = w.nq, nk = w.nk, qt = w.qt, n = w.n, off = w.off;
+      if (n == 0) {
+        // No row of this tile sees a key (bottom-right with nq > nk, or a
+        // sequence without keys): the softmax is empty, O = 0 and LSE = log 0.
+        const int rows = nq - qt * kTile < kTile ? nq - qt * kTile : kTile;
+        const size_t grow0 = static_cast<size_t>(z) * Nq + q0 + static_cast<size_t>(qt) * kTile;
+        const int t0 = static_cast<int>(threadIdx.x) - 128;  // the 256 softmax threads
+        for (int e = t0; e < rows * D / 8; e += 256)
+          reinterpret_cast<uint4*>(o_ptr + grow0 * D)[e] = make_uint4(0u, 0u, 0u, 0u);
+        for (int e = t0; e < rows; e += 256) lse_ptr[grow0 + e] = -INFINITY;
+        continue;
+      }
+      if (!q_ready) ok = copy_q(uu & 1);
+      q_ready = false;
 
       float m_run = -INFINITY;  // running row max (log2 units; stale by < 8)
       float l_run = 0.f;        // this warpgroup's part of sum exp2(score - m_run)
@@ -607,6 +613,23 @@ __global__ void __launch_bounds__(384, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_full[b]);
+      }
+      // With early_q (grids of short query rows) the next unit's Q goes
+      // into tensor memory now, before this unit's epilogue: every S product
+      // of this unit (the readers of the old Q) has been consumed, and the
+      // MMA warp can start the next unit's first two S products while the
+      // epilogue runs (d <= 128; at d = 256 the next Q is loaded only once
+      // this unit's products are done).
+      if constexpr (!L::kWide) {
+        for (int r2 = r + 1; early_q && ok && r2 < slots; ++r2) {
+          const int u2 = unit_index(r2);
+          if (u2 < 0) continue;
+          const Unit w2 = unit_of(u2);
+          if (!w2.live || w2.n == 0) continue;
+          ok = copy_q((uu + 1) & 1);
+          q_ready = true;
+          break;
+        }
       }
       // Epilogue: combine the two warpgroups' row sums, then each warpgroup
       // writes its half of the head dimension of O.
