@@ -236,14 +236,9 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   // Causal grids with at least two units per CTA deal heavy and light tiles
   // out in pairs (tile_order.h).
   const int fold = CAUSAL && units >= 2u * sms ? 1 : 0;
-  // Short query rows (few key tiles per unit) copy the next unit's Q before
-  // the epilogue, so that its first products overlap the epilogue; long
-  // causal rows measured faster without it.
-  const double tiles_per_unit = CAUSAL ? 0.5 * (pb.ktiles + 1) : static_cast<double>(pb.ktiles);
-  const int early_q = tiles_per_unit <= 16.0 ? 1 : 0;
   kern<<<grid, 384, L::kAlloc, st>>>(mq, mk, mv, mo, static_cast<uint16_t*>(o), lse, pb.cu_q, pb.cu_k, pb.H, pb.rows_q,
                                      pb.rows_k, pb.bottom_right, scale_log2, pb.problems, pb.qtiles, group, fold,
-                                     early_q, o_scale);
+                                     o_scale);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -37,6 +37,11 @@
 // registers, dQ(j) once they have written dS(j), dP(j+1) behind dQ(j) (which
 // reads the dS it overwrites).  The warps find S(j+1) ready when they finish
 // tile j and wait for dP(j+1) only while dQ(j) and dP(j+1) run.
+// d = 256 (the only dQ kernel of the d = 256 backward): key tiles of 64 rows
+// (each warpgroup owns 32 key columns), S in [0, 64), dP in [64, 128), the
+// dQ accumulator in [128, 384) and Q in [384, 512); dO has no room in tensor
+// memory and stays in shared memory, so dP reads both operands from there.
+// Once Q is in tensor memory its staging area holds two more ring slots.
 #pragma once
 
 #include "sm100.cuh"

@@ -87,7 +87,12 @@ struct FwdLayout {
   // xmax[2], xsum, o_free, o_staged
   static constexpr int kNumBars = 2 + 2 * kSlots + 12;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16;
+  // The CTA's first kTabSlots work units, decoded once at set-up (two int4
+  // per slot; see unit_of), so that no role spends the time at a tile
+  // boundary on the integer divisions of the decode.
+  static constexpr int kTabSlots = 256;
+  static constexpr int kTabOff = kMiscOff + 16;
+  static constexpr int kBytes = kTabOff + kTabSlots * 32;
   static constexpr int kAlloc = kBytes + 1024 <= 232448 ? kBytes + 1024 : 232448;
   static_assert(kBytes <= 232448, "shared memory budget");
   // Tensor-memory columns.  d = 256: the two S buffers and O take all 512
@@ -114,7 +119,7 @@ __global__ void __launch_bounds__(384, 1)
                uint16_t* __restrict__ o_ptr,
                float* __restrict__ lse_ptr, const int* __restrict__ cu_q, const int* __restrict__ cu_k, int H,
                int Nq, int Nk, int bottom_right, float scale_log2, int problems, int grid_tiles, int group,
-               int fold, int early_q, float o_scale) {
+               int fold, float o_scale) {
   static_assert(!F8 || BF16, "the 8-bit forward writes bf16");
   using L = FwdLayout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
@@ -196,6 +201,24 @@ __global__ void __launch_bounds__(384, 1)
     }
     return w;
   };
+  // Slot r's unit: false for an empty slot.  Slots below kTabSlots come from
+  // the table (n = -1 marks a unit past the end of a shorter sequence, -2 an
+  // empty slot), later ones are decoded here.
+  int4* tab = reinterpret_cast<int4*>(smem + L::kTabOff);
+  auto slot_unit = [&](int r, Unit& w) {
+    if (r < L::kTabSlots) {
+      const int4 a = tab[2 * r], c = tab[2 * r + 1];
+      if (c.z == -2) return false;
+      w.z = a.x; w.q0 = a.y; w.k0 = a.z; w.nq = a.w;
+      w.nk = c.x; w.qt = c.y; w.n = c.z < 0 ? 0 : c.z; w.off = c.w;
+      w.live = c.z != -1;
+      return true;
+    }
+    const int u = unit_index(r);
+    if (u < 0) return false;
+    w = unit_of(u);
+    return true;
+  };
 
   // Refuse to run (and report) if alignment left too little shared memory.
   if (static_cast<uint32_t>(smem - smem_raw) + L::kBytes > dynamic_smem_bytes()) {
@@ -234,6 +257,18 @@ __global__ void __launch_bounds__(384, 1)
     uint4* ones = reinterpret_cast<uint4*>(smem + L::kOnesOff);
     for (int i = lane; i < L::kOnesBytes / 16; i += 32) ones[i] = make_uint4(one2, one2, one2, one2);
     fence_proxy_async_smem();
+    // The unit table.
+    const int n_tab = slots < L::kTabSlots ? slots : L::kTabSlots;
+    for (int r = lane; r < n_tab; r += 32) {
+      const int u = unit_index(r);
+      if (u < 0) {
+        tab[2 * r + 1] = make_int4(0, 0, -2, 0);
+        continue;
+      }
+      const Unit w = unit_of(u);
+      tab[2 * r] = make_int4(w.z, w.q0, w.k0, w.nq);
+      tab[2 * r + 1] = make_int4(w.nk, w.qt, w.live ? w.n : -1, w.off);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -250,10 +285,8 @@ __global__ void __launch_bounds__(384, 1)
       int uu = 0;    // units with key tiles whose Q load was issued
       bool ok = true;
       for (int r = 0; ok && r < slots; ++r) {
-        const int u = unit_index(r);
-        if (u < 0) continue;
-        const Unit w = unit_of(u);
-        if (!w.live || w.n == 0) continue;
+        Unit w;
+        if (!slot_unit(r, w) || !w.live || w.n == 0) continue;
         // The Q buffer is free once the previous unit's Q has been copied
         // into tensor memory (d = 256: once its S products are done).
         if (uu > 0 && !(ok = mbar_wait(L::kWide ? o_full : q_tmem, (uu - 1) & 1, abort_flag))) break;
@@ -355,10 +388,8 @@ __global__ void __launch_bounds__(384, 1)
     int uu = 0, g = 0;  // units with key tiles, key tiles before the current unit
     bool ok = true;
     for (int r = 0; ok && r < slots; ++r) {
-      const int u = unit_index(r);
-      if (u < 0) continue;
-      const Unit w = unit_of(u);
-      if (!w.live || w.n == 0) continue;
+      Unit w;
+      if (!slot_unit(r, w) || !w.live || w.n == 0) continue;
       const int n = w.n;
       // Q of this unit is in tensor memory (d = 256: in shared memory).
       if (!(ok = wait_all(q_tmem, uu & 1))) break;
@@ -453,10 +484,8 @@ __global__ void __launch_bounds__(384, 1)
     bool q_ready = false;  // the next unit's Q is already in tensor memory
     bool ok = true;
     for (int r = 0; ok && r < slots; ++r) {
-      const int u = unit_index(r);
-      if (u < 0) continue;
-      const Unit w = unit_of(u);
-      if (!w.live) continue;
+      Unit w;
+      if (!slot_unit(r, w) || !w.live) continue;
       const int z = w.z, q0 = w.q0, nq = w.nq, nk = w.nk, qt = w.qt, n = w.n, off = w.off;
       if (n == 0) {
         // No row of this tile sees a key (bottom-right with nq > nk, or a
@@ -614,18 +643,15 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_before();
         mbar_arrive(&p_full[b]);
       }
-      // With early_q (grids of short query rows) the next unit's Q goes
-      // into tensor memory now, before this unit's epilogue: every S product
-      // of this unit (the readers of the old Q) has been consumed, and the
-      // MMA warp can start the next unit's first two S products while the
-      // epilogue runs (d <= 128; at d = 256 the next Q is loaded only once
-      // this unit's products are done).
+      // The next unit's Q goes into tensor memory now, before this unit's
+      // epilogue: every S product of this unit (the readers of the old Q)
+      // has been consumed, and the MMA warp can start the next unit's first
+      // two S products while the epilogue runs (d <= 128; at d = 256 the
+      // next Q is loaded only once this unit's products are done).
       if constexpr (!L::kWide) {
-        for (int r2 = r + 1; early_q && ok && r2 < slots; ++r2) {
-          const int u2 = unit_index(r2);
-          if (u2 < 0) continue;
-          const Unit w2 = unit_of(u2);
-          if (!w2.live || w2.n == 0) continue;
+        for (int r2 = r + 1; ok && r2 < slots; ++r2) {
+          Unit w2;
+          if (!slot_unit(r2, w2) || !w2.live || w2.n == 0) continue;
           ok = copy_q((uu + 1) & 1);
           q_ready = true;
           break;
