@@ -25,12 +25,16 @@
 // CTA layout (384 threads, one CTA per SM):
 //   warp 0       TMA producer: per query tile Q, then K_0, K_1, V_0, K_2,
 //                V_1, ... through a ring of shared-memory slots
-//   warp 1       MMA issuer (one thread)
+//   warp 1       MMA issuer (one elected lane per group)
 //   warp 2       tensor-memory allocation / release
+//   warp 3       set-up: the ones tile and the table of decoded work units
 //   warps 4-7    softmax for key columns [0, 64) of every key tile
 //   warps 8-11   softmax for key columns [64, 128)
 //                (thread = query row = TMEM lane; the two warpgroups
-//                exchange their partial row maxima through shared memory)
+//                exchange their partial row maxima through shared memory,
+//                copy each query tile's Q into tensor memory -- the next
+//                tile's before this one's epilogue -- and write O through a
+//                shared-memory staging tile and TMA stores)
 //
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   [0, D/2)     Q, 16-bit pairs (A operand of S = Q K^T)

@@ -252,3 +252,21 @@ def test_causal_sweep_workload_sampled(n):
     for s, ref, lref in zip(slices, refs, lrefs):
         parity.assert_o(parity.f64(of[s][rows]), ref, q.dtype, f"{w.label()} slice {s}")
         parity.assert_lse(parity.f64(lf[s][rows]), lref, f"{w.label()} slice {s}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_forward_grid_past_the_unit_table(causal):
+    """A grid with more work units per CTA than the kernel's set-up table
+    holds (256): B64 H32 N2368 d64 is 38,912 query tiles, 263 slots per CTA
+    on 148 SMs, so the last units of every CTA are decoded on the fly.
+    Those are the last problems of the launch order; slices from the first
+    and the last launch group are checked in full against the oracle."""
+    B, H, N, d = 64, 32, 2368, 64
+    q, k, v = draw(B, H, N, N, d, torch.float16, seed=991 + int(causal))
+    o, lse = run_forward(q, k, v, causal, 0.125)
+    slices = [0, B * H - 2, B * H - 1]
+    refs, lrefs = parity.oracle_forward_slices(q, k, v, 0.125, causal, slices)
+    of, lf = o.reshape(B * H, N, d), lse.reshape(B * H, N)
+    for s, ref, lref in zip(slices, refs, lrefs):
+        parity.assert_o(parity.f64(of[s]), ref, q.dtype, f"unit-table overflow causal={causal} slice {s}")
+        parity.assert_lse(parity.f64(lf[s]), lref, f"unit-table overflow causal={causal} slice {s}")
