@@ -22,9 +22,11 @@
 // K-major A of S and dP and the MN-major A of dK^T and dV^T; P and dS go
 // from the softmax warps to shared memory as the MN-major B operands.
 // Shared memory holds one Q_i and one dO_i (64 KB each), so the next query
-// tile's dO is loaded once dV^T has read this one, and its Q once dK^T has;
-// per query tile the issue order is dP, S, dV^T, dK^T, which lets dP(i+1)
-// run while Q_{i+1} is in flight.
+// tile's Q is loaded once dK^T has read this one, and its dO once dV^T has.
+// The next S product, which starts the next tile's softmax, waits for that Q
+// load; so per query tile the issue order is S, dP, dK^T, dV^T: dK^T, the
+// last reader of Q_i, goes first once dS is written (P is ready earlier, but
+// dV^T can wait), and dV^T then runs while Q_{i+1} is in flight.
 //
 // CTA layout (384 threads, one CTA per SM):
 //   warp 0       TMA producer: K_j and V_j once; dO_i, Q_i per query tile
@@ -204,16 +206,16 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = true;
       for (int it = 0; it < n_it; ++it) {
         const int row0 = q0 + (i0 + it) * kQR;
-        if (it > 0 && !(ok = mbar_wait(do_free, (it - 1) & 1, abort_flag))) break;
-        mbar_arrive_expect_tx(do_full, L::kQTileBytes);
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(smem + L::kDOOff + c * L::kQChunkBytes, &tm_do, do_full, c * 64, row0, z);
-        ++n_do;
         if (it > 0 && !(ok = mbar_wait(q_free, (it - 1) & 1, abort_flag))) break;
         mbar_arrive_expect_tx(q_full, L::kQTileBytes);
         for (int c = 0; c < L::kChunks; ++c)
           tma_load_3d(smem + L::kQOff + c * L::kQChunkBytes, &tm_q, q_full, c * 64, row0, z);
         ++n_q;
+        if (it > 0 && !(ok = mbar_wait(do_free, (it - 1) & 1, abort_flag))) break;
+        mbar_arrive_expect_tx(do_full, L::kQTileBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(smem + L::kDOOff + c * L::kQChunkBytes, &tm_do, do_full, c * 64, row0, z);
+        ++n_do;
       }
       if (!ok) {
         // Let the copies already issued land before the CTA exits.
@@ -259,15 +261,6 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = wait_all(kv_full, 0);
     for (int it = 0; ok && it < n_it; ++it) {
       const uint32_t par = it & 1, prev = (it - 1) & 1;
-      // dP(it) = dO_i V_j^T over dP(it-1), which the softmax warps have loaded.
-      if (!(ok = wait_all(do_full, par))) break;
-      if (it > 0 && !(ok = wait_all(dp_read, prev))) break;
-      tc_fence_after();
-      if (elect_one()) {
-        issue_qk(L::kColDP, L::kDOOff, L::kVOff);
-        mma_commit(dp_full);
-      }
-      __syncwarp();
       // S(it) = Q_i K_j^T.
       if (!(ok = wait_all(q_full, par))) break;
       if (it > 0 && !(ok = wait_all(s_read, prev))) break;
@@ -277,13 +270,13 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(s_full);
       }
       __syncwarp();
-      // dV^T += dO_i^T P(it): then dO_i and P are free.
-      if (!(ok = wait_all(p_full, par))) break;
+      // dP(it) = dO_i V_j^T over dP(it-1), which the softmax warps have loaded.
+      if (!(ok = wait_all(do_full, par))) break;
+      if (it > 0 && !(ok = wait_all(dp_read, prev))) break;
       tc_fence_after();
       if (elect_one()) {
-        issue_acc(L::kColDV, L::kDOOff, L::kPOff, it == 0);
-        mma_commit(p_free);
-        mma_commit(do_free);
+        issue_qk(L::kColDP, L::kDOOff, L::kVOff);
+        mma_commit(dp_full);
       }
       __syncwarp();
       // dK^T += Q_i^T dS(it): then Q_i and dS are free.
@@ -293,6 +286,15 @@ __global__ void __launch_bounds__(384, 1)
         issue_acc(L::kColDK, L::kQOff, L::kDSOff, it == 0);
         mma_commit(ds_free);
         mma_commit(q_free);
+      }
+      __syncwarp();
+      // dV^T += dO_i^T P(it): then dO_i and P are free.
+      if (!(ok = wait_all(p_full, par))) break;
+      tc_fence_after();
+      if (elect_one()) {
+        issue_acc(L::kColDV, L::kDOOff, L::kPOff, it == 0);
+        mma_commit(p_free);
+        mma_commit(do_free);
         if (it == n_it - 1) mma_commit(acc_done);
       }
       __syncwarp();
