@@ -154,3 +154,20 @@ def test_sample_parity_non_finite_output_stays_strict_json():
     out = bench.sample_parity(w, ref, o, lse, None)
     assert out["o_max_abs_err"] == "non-finite" and out["within_tol"] is False
     json.dumps(out, allow_nan=False)
+
+
+def test_l2_flush_rule_follows_the_input_size():
+    """Workloads whose inputs fit the 126 MB L2 are timed with a flush before
+    every step and say so; larger ones are not, and say that instead."""
+    from exact_attention_150_b200 import workloads
+    small = [workloads.TINY, workloads.SWEEP[512], workloads.SWEEP[1024], workloads.TRAIN_D64]
+    large = [workloads.LONG_CTX, workloads.LAYER_7B, workloads.CAUSAL_SWEEP[4096], workloads.LONG_CTX_D256]
+    for w in small:
+        assert bench.needs_flush(w), w.name
+        assert bench.config_of(w, 1)["l2"].startswith("flush:"), w.name
+    for w in large:
+        assert not bench.needs_flush(w), w.name
+        assert bench.config_of(w, 1)["l2"].startswith("no flush:"), w.name
+    # The rule counts the inputs one step reads: Q, K, V, and dO with a backward.
+    assert bench.step_input_bytes(workloads.TRAIN_D64) == 4 * 2 * 16 * 4096 * 64 * 2
+    assert bench.step_input_bytes(workloads.LAYER_7B) == 3 * 4 * 32 * 2048 * 128 * 2
