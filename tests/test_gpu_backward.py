@@ -283,10 +283,11 @@ def test_deterministic_backward_is_bit_reproducible(causal):
 # ------------------------------------------------- fp16 range of the row terms
 #
 # The backward adds -LSE_i / scale and -D_i to its fp32 products as 16-bit
-# pieces.  In fp16 a single piece overflows past 65504; these cases all have
-# terms beyond that and must still match the oracle.
+# pieces (d <= 128).  In fp16 a single piece overflows past 65504; these cases
+# all have terms beyond that and must still match the oracle.  At d = 256 the
+# terms are per-thread fp32 values; the same cases check that there too.
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal,nq,nk", [(True, 777, 777), ("bottom_right", 300, 900)])
 @pytest.mark.parametrize("scale", [1e-4, 1e-5, -1e-4])
 def test_backward_fp16_small_scale(scale, causal, nq, nk, d):
