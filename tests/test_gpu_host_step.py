@@ -35,6 +35,7 @@ def _device_path(q, k, v, do, causal, scale):
     (2, 3, 301, 257, 64, torch.float16, False, 4),        # odd Nq, B > 1, 6 slices in chunks of 2
     (2, 3, 129, 300, 128, torch.float16, "bottom_right", 5),
     (1, 2, 640, 640, 64, torch.bfloat16, True, 1),
+    (1, 4, 300, 300, 256, torch.bfloat16, True, 2),       # head dimension 256
 ])
 def test_host_step_matches_device_path(B, H, nq, nk, d, dtype, causal, chunks):
     q, k, v, do = draw(B, H, nq, nk, d, dtype, 4000 + nq + nk, with_grad=True)
